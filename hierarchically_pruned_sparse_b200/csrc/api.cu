@@ -1,0 +1,286 @@
+// C ABI of libhip_sparse.so: argument validation, launch planning, dispatch.
+// Every entry point validates on the host before launching anything and
+// launches only on params->stream; nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "hip_sparse.h"
+#include "hips_common.cuh"
+#include "hips_kernels.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kPlanSMs = 148;         // B200 streaming multiprocessors
+constexpr size_t kStatusBytes = 256;  // head of every workspace
+constexpr int kMaxSmem = 227 * 1024;
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int validate(const hips_params* p, int op) {
+  if (!p) return HIPS_ERR_INVALID_ARG;
+  if (p->batch <= 0 || p->n_qheads <= 0 || p->n_kvheads <= 0) return HIPS_ERR_INVALID_ARG;
+  if (p->n_qheads % p->n_kvheads) return HIPS_ERR_INVALID_ARG;
+  if (p->head_dim != hips::kD) return HIPS_ERR_UNSUPPORTED;
+  if (p->dtype != HIPS_F32 && p->dtype != HIPS_BF16) return HIPS_ERR_UNSUPPORTED;
+  if (p->reserved != 0) return HIPS_ERR_INVALID_ARG;
+  if (p->seq_len <= 0 || p->seq_len >= (int64_t{1} << 31)) return HIPS_ERR_INVALID_ARG;
+  if (p->kv_capacity < p->seq_len) return HIPS_ERR_INVALID_ARG;
+  if (p->q_len <= 0 || p->q_pos0 < 0 || p->q_pos0 + p->q_len > p->seq_len) return HIPS_ERR_INVALID_ARG;
+  if (op != HIPS_OP_DENSE) {
+    if (p->mask_len <= 0 || p->mask_len > p->seq_len) return HIPS_ERR_INVALID_ARG;
+    if (p->block_q <= 0 || !is_pow2(p->block_k)) return HIPS_ERR_INVALID_ARG;
+    if (p->topk < p->block_k || p->topk % p->block_k) return HIPS_ERR_INVALID_ARG;
+    if (p->sink < 0 || p->window < 0) return HIPS_ERR_INVALID_ARG;
+    if (p->topk / p->block_k > hips::kMaxN0) return HIPS_ERR_UNSUPPORTED;
+  }
+  const double elems = static_cast<double>(p->batch) * p->n_kvheads * p->kv_capacity * p->head_dim;
+  if (elems > 4.0e18) return HIPS_ERR_INVALID_ARG;
+  return HIPS_OK;
+}
+
+int64_t row_stride(const hips_params* p) {
+  const int64_t bk = p->block_k;
+  int64_t cap = p->topk / bk + cdiv(p->sink, bk);
+  if (p->window > 0) cap += cdiv(static_cast<int64_t>(p->window) + p->block_q - 1, bk) + 1;
+  return 1 + cap;
+}
+
+int group_rows(const hips_params* p, int block_q) {
+  return (p->n_qheads / p->n_kvheads) * std::min(block_q, p->q_len);
+}
+
+// ---------------------------------------------------------------- mask plan
+
+struct MaskPlan {
+  hips::MaskArgs a;
+  int smem;
+  size_t ws;
+};
+
+int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
+  hips::MaskArgs& a = plan->a;
+  a = hips::MaskArgs{};
+  a.dtype = p->dtype;
+  a.n_qheads = p->n_qheads;
+  a.n_kvheads = p->n_kvheads;
+  a.group = p->n_qheads / p->n_kvheads;
+  a.q_len = p->q_len;
+  a.block_q = p->block_q;
+  a.block_k = p->block_k;
+  a.n0max = p->topk / p->block_k;
+  a.sink = p->sink;
+  a.window = p->window;
+  a.nqb = static_cast<int>(cdiv(p->q_len, p->block_q));
+  a.units = static_cast<int64_t>(p->batch) * p->n_kvheads * a.nqb;
+  a.seq_len = p->seq_len;
+  a.kv_cap = p->kv_capacity;
+  a.q_pos0 = p->q_pos0;
+  a.row_stride = row_stride(p);
+  a.rows_max = group_rows(p, p->block_q);
+  if (a.rows_max > 32 || a.units > 65535) return HIPS_ERR_UNSUPPORTED;
+  const int rc = hips::mask_fma_rc(a.rows_max);
+  a.rows_pad = static_cast<int>(cdiv(a.rows_max, rc) * rc);
+  const int tile_keys = hips::mask_fma_tile_keys(p->dtype);
+  if (p->block_k > tile_keys) return HIPS_ERR_UNSUPPORTED;
+  const int cpt = tile_keys / p->block_k;
+  const int64_t ncand = 2 * static_cast<int64_t>(a.n0max);
+  int c = 1;
+  while (c < cluster_cap && a.units * (2 * c) <= kPlanSMs && cdiv(ncand, 2 * c) >= cpt) c *= 2;
+  a.cluster = c;
+  a.per_cta = static_cast<int>(cdiv(ncand, c));
+  plan->smem = hips::mask_fma_smem_bytes(a.n0max, a.rows_pad, a.per_cta);
+  if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
+  plan->ws = kStatusBytes;
+  return HIPS_OK;
+}
+
+// ---------------------------------------------------------------- attention plan
+
+struct AttnPlan {
+  hips::AttnArgs a;
+  int smem;
+  size_t ws;
+};
+
+int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
+  hips::AttnArgs& a = plan->a;
+  a = hips::AttnArgs{};
+  const int block_q = dense ? 1 : p->block_q;
+  a.dtype = p->dtype;
+  a.batch = p->batch;
+  a.n_qheads = p->n_qheads;
+  a.n_kvheads = p->n_kvheads;
+  a.group = p->n_qheads / p->n_kvheads;
+  a.q_len = p->q_len;
+  a.block_q = block_q;
+  a.nqb = static_cast<int>(cdiv(p->q_len, block_q));
+  a.dense = dense ? 1 : 0;
+  a.rows_max = group_rows(p, block_q);
+  a.seq_len = p->seq_len;
+  a.mask_len = dense ? p->seq_len : p->mask_len;
+  a.kv_cap = p->kv_capacity;
+  a.q_pos0 = p->q_pos0;
+  a.row_stride = dense ? 0 : row_stride(p);
+  a.rows_total = static_cast<int64_t>(p->batch) * p->n_qheads * p->q_len;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
+  if (a.rows_max > 8) return HIPS_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(a.nqb) * p->n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
+  a.item_keys = dense ? 16 : p->block_k;
+  const int tile_keys = hips::attn_fma_tile_keys(p->dtype);
+  if (a.item_keys > tile_keys) return HIPS_ERR_UNSUPPORTED;
+  const int ipt = tile_keys / a.item_keys;
+  int64_t w_max;
+  if (dense) {
+    w_max = cdiv(std::min<int64_t>(p->q_pos0 + p->q_len, p->seq_len), a.item_keys);
+  } else {
+    w_max = (a.row_stride - 1) + cdiv(std::max<int64_t>(0, p->seq_len - p->mask_len), a.item_keys);
+  }
+  const int64_t units = static_cast<int64_t>(p->batch) * p->n_kvheads * a.nqb;
+  int64_t nsplit = std::min<int64_t>(cdiv(2 * kPlanSMs, units), cdiv(w_max, ipt));
+  nsplit = std::max<int64_t>(1, std::min<int64_t>(nsplit, 1024));
+  a.nsplit = static_cast<int>(nsplit);
+  a.table_items = dense ? 0 : static_cast<int>(cdiv(w_max, nsplit));
+  plan->smem = hips::attn_fma_smem_bytes(p->dtype, a.rows_max, a.table_items);
+  if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
+  size_t part = 0;
+  if (a.nsplit > 1) part = static_cast<size_t>(a.rows_total) * a.nsplit * (hips::kD + 2) * sizeof(float);
+  plan->ws = kStatusBytes + (part + 255) / 256 * 256;
+  return HIPS_OK;
+}
+
+int check_workspace(const hips_params* p, size_t need) {
+  if (!p->workspace || !aligned(p->workspace, 256) || p->workspace_bytes < need)
+    return HIPS_ERR_WORKSPACE;
+  return HIPS_OK;
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return HIPS_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return HIPS_ERR_CUDA;
+}
+
+int run_attention(const void* q, const void* k, const void* v, const int32_t* idx,
+                  const hips_params* p, void* out, bool dense) {
+  int st = validate(p, dense ? HIPS_OP_DENSE : HIPS_OP_SPARSE);
+  if (st) return st;
+  if (!q || !k || !v || !out || (!dense && !idx)) return HIPS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (idx && !aligned(idx, 4)))
+    return HIPS_ERR_INVALID_ARG;
+  AttnPlan plan;
+  st = plan_attn(p, dense, &plan);
+  if (st) return st;
+  st = check_workspace(p, plan.ws);
+  if (st) return st;
+  hips::AttnArgs& a = plan.a;
+  a.q = q; a.k = k; a.v = v; a.idx = idx; a.out = out;
+  a.status = static_cast<hips::Status*>(p->workspace);
+  a.part = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + kStatusBytes);
+  return cuda_status(hips::launch_attn_fma(a, plan.smem, static_cast<cudaStream_t>(p->stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t hip_idx_row_stride(const hips_params* params) {
+  if (validate(params, HIPS_OP_MASK) != HIPS_OK) return 0;
+  return row_stride(params);
+}
+
+size_t hip_workspace_size(const hips_params* params, int op) {
+  if (validate(params, op) != HIPS_OK) return 0;
+  if (op == HIPS_OP_MASK) {
+    MaskPlan plan;
+    return plan_mask(params, 16, &plan) == HIPS_OK ? plan.ws : 0;
+  }
+  if (op == HIPS_OP_SPARSE || op == HIPS_OP_DENSE) {
+    AttnPlan plan;
+    return plan_attn(params, op == HIPS_OP_DENSE, &plan) == HIPS_OK ? plan.ws : 0;
+  }
+  return 0;
+}
+
+int hip_workspace_init(const hips_params* params) {
+  if (!params || !params->workspace || params->workspace_bytes < kStatusBytes) return HIPS_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(params->workspace, 0, kStatusBytes,
+                                     static_cast<cudaStream_t>(params->stream)));
+}
+
+int hip_check_status(const hips_params* params) {
+  if (!params || !params->workspace || params->workspace_bytes < kStatusBytes) return HIPS_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(params->stream);
+  hips::Status host{};
+  int st = cuda_status(cudaStreamSynchronize(s));
+  if (st) return st;
+  st = cuda_status(cudaMemcpy(&host, params->workspace, sizeof(host), cudaMemcpyDeviceToHost));
+  if (st) return st;
+  if (host.flags == 0) return HIPS_OK;
+  st = cuda_status(cudaMemset(params->workspace, 0, kStatusBytes));
+  if (st) return st;
+  return HIPS_ERR_TIMEOUT;
+}
+
+int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* idx_out) {
+  int st = validate(params, HIPS_OP_MASK);
+  if (st) return st;
+  if (!q || !k || !idx_out) return HIPS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx_out, 4)) return HIPS_ERR_INVALID_ARG;
+  MaskPlan plan;
+  st = plan_mask(params, 16, &plan);
+  if (st) return st;
+  st = check_workspace(params, plan.ws);
+  if (st) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
+  // A 16-CTA cluster needs 16 free SMs of one GPC; fall back to smaller
+  // clusters if the device refuses the shape.
+  for (int cap = 16; cap >= 1; cap /= 2) {
+    st = plan_mask(params, cap, &plan);
+    if (st) return st;
+    if (plan.a.cluster > cap) continue;
+    hips::MaskArgs& a = plan.a;
+    a.q = q; a.k = k; a.idx = idx_out;
+    a.status = static_cast<hips::Status*>(params->workspace);
+    const cudaError_t e = hips::launch_mask_fma(a, plan.smem, stream);
+    if (e == cudaSuccess) return HIPS_OK;
+    if ((e == cudaErrorInvalidClusterSize || e == cudaErrorLaunchOutOfResources) && cap > 1) {
+      (void)cudaGetLastError();
+      continue;
+    }
+    return cuda_status(e);
+  }
+  return HIPS_ERR_UNSUPPORTED;
+}
+
+int hip_sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx,
+                    const hips_params* params, void* out) {
+  return run_attention(q, k, v, idx, params, out, false);
+}
+
+int hip_dense_attn(const void* q, const void* k, const void* v, const hips_params* params,
+                   void* out) {
+  return run_attention(q, k, v, nullptr, params, out, true);
+}
+
+int hip_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* hip_error_string(int status) {
+  switch (status) {
+    case HIPS_OK: return "ok";
+    case HIPS_ERR_INVALID_ARG: return "invalid argument";
+    case HIPS_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case HIPS_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case HIPS_ERR_CUDA: return "CUDA launch failed";
+    case HIPS_ERR_TIMEOUT: return "a bounded device wait expired";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,381 @@
+// Block-sparse (and dense) attention on CUDA cores for decode-sized query
+// groups, split over the key list (flash-decoding) plus a combine kernel.
+//
+// The sparse attention step consumes, per query block, the ascending list of
+// selected key blocks and its nnz ("A Training-free Sub-quadratic Cost
+// Transformer Model Serving Framework With Hierarchically Pruned Attention",
+// Author Rebuttal to the Reviewer NLBm, W2). A query row at position p
+// attends the keys j <= p of those blocks that lie below mask_len, plus every
+// key in [mask_len, seq_len) appended since the mask was computed (the mask
+// refresh interval r_m of the research-map summary, Limitations).
+//
+// Design: grid (splits, KV head x query block, sequence). A split takes a
+// contiguous range of work items (one key block each); K and V rows of a
+// 64-key tile are gathered with bulk async copies into a 3-stage ring, the
+// G query heads of the group share every gathered tile, and each of 8 warps
+// works on 4 keys at a time with 8 lanes per key (16 head elements per lane).
+// Scores go through an fp32 online softmax (exp2 domain); each split writes
+// (m, l, unnormalised o) and the combine kernel merges the splits.
+#include "hips_common.cuh"
+#include "hips_kernels.h"
+
+namespace hips {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kTileBytes = 16384;  // one of K or V per stage
+
+struct AttnSmem {
+  int kring, vring, bars, table, s, p, alpha, ml, total;
+};
+
+__host__ __device__ inline int align16(int x) { return (x + 15) / 16 * 16; }
+
+__host__ __device__ inline AttnSmem attn_smem_layout(int tile_keys, int rc, int table_items) {
+  AttnSmem L;
+  int o = 0;
+  L.kring = o;  o += kStages * kTileBytes;
+  L.vring = o;  o += kStages * kTileBytes;
+  L.bars = o;   o += align16(kStages * 8);
+  L.table = o;  o += align16(table_items * 8);
+  L.s = o;      o += align16(rc * tile_keys * 4);
+  L.p = o;      o += align16(rc * tile_keys * 4);
+  L.alpha = o;  o += align16(rc * 4);
+  L.ml = o;     o += align16(2 * rc * 4);
+  L.total = o;
+  return L;
+}
+
+template <typename T, int RC>
+__global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int kRowB = row_bytes<T>();
+  constexpr int kTileKeys = kTileBytes / kRowB;
+  constexpr int kPasses = kTileKeys / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane8 = lane & 7, grp = lane >> 3;
+
+  const int split = blockIdx.x;
+  const int qb = blockIdx.y % a.nqb;
+  const int g = blockIdx.y / a.nqb;
+  const int b = blockIdx.z;
+  const int i0 = qb * a.block_q;
+  const int nrows = min(a.block_q, a.q_len - i0);
+  const int R = a.group * nrows;
+  const int64_t q_first = a.q_pos0 + i0, q_last = q_first + nrows - 1;
+  const int IK = a.item_keys;
+
+  const AttnSmem L = attn_smem_layout(kTileKeys, RC, a.table_items);
+  unsigned char* kring = smem + L.kring;
+  unsigned char* vring = smem + L.vring;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  int2* table = reinterpret_cast<int2*>(smem + L.table);
+  float* s_sm = reinterpret_cast<float*>(smem + L.s);
+  float* p_sm = reinterpret_cast<float*>(smem + L.p);
+  float* alpha_sm = reinterpret_cast<float*>(smem + L.alpha);
+  float* ml_sm = reinterpret_cast<float*>(smem + L.ml);
+
+  // ---- work items of this unit and this split's range
+  const int64_t unit = (static_cast<int64_t>(b) * a.n_kvheads + g) * a.nqb + qb;
+  const int32_t* idx_row = a.dense ? nullptr : a.idx + unit * a.row_stride;
+  int64_t nitems;
+  int nnz = 0;
+  if (a.dense) {
+    const int64_t Tc = min(q_last + 1, a.seq_len);
+    nitems = (Tc + IK - 1) / IK;
+  } else {
+    nnz = max(0, min(idx_row[0], static_cast<int>(a.row_stride - 1)));
+    const int64_t tail = max64(0, a.seq_len - a.mask_len);
+    nitems = nnz + (tail + IK - 1) / IK;
+  }
+  const int64_t per = (nitems + a.nsplit - 1) / a.nsplit;
+  const int64_t it_lo = min(nitems, split * per), it_hi = min(nitems, it_lo + per);
+  const int nmine = static_cast<int>(it_hi - it_lo);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  // item table (sparse): first key and key count of every item of this split;
+  // ids read from idx are range-checked so a malformed row cannot drive reads
+  // outside [0, seq_len)
+  const int64_t vis = min64(q_last + 1, a.seq_len);
+  if (!a.dense) {
+    for (int t = tid; t < nmine; t += kThreads) {
+      const int64_t it = it_lo + t;
+      int64_t j0, n;
+      if (it < nnz) {
+        const int64_t c = idx_row[1 + it];
+        j0 = c * IK;
+        n = c < 0 ? 0 : min64(IK, min64(a.mask_len, vis) - j0);
+      } else {
+        j0 = a.mask_len + (it - nnz) * IK;
+        n = min64(IK, vis - j0);
+      }
+      table[t] = make_int2(static_cast<int>(max64(j0, 0)), static_cast<int>(max64(n, 0)));
+    }
+  }
+  auto item_at = [&](int t) -> int2 {
+    if (!a.dense) return table[t];
+    const int64_t j0 = (it_lo + t) * IK;
+    return make_int2(static_cast<int>(j0), static_cast<int>(max64(min64(IK, vis - j0), 0)));
+  };
+  __syncthreads();
+
+  // query rows in registers: lane holds 16 elements of each of the RC rows
+  float qreg[RC][16];
+  {
+    const T* qp = static_cast<const T*>(a.q);
+#pragma unroll
+    for (int r = 0; r < RC; ++r) {
+      if (r < R) {
+        const int h = g * a.group + r / nrows, i = i0 + r % nrows;
+        const unsigned char* row = reinterpret_cast<const unsigned char*>(
+            qp + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i) * kD);
+        load_row16<T>(row, lane8, qreg[r]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) qreg[r][e] = 0.0f;
+      }
+    }
+  }
+
+  const size_t plane = (static_cast<size_t>(b) * a.n_kvheads + g) * static_cast<size_t>(a.kv_cap) * kRowB;
+  const unsigned char* kbase = static_cast<const unsigned char*>(a.k) + plane;
+  const unsigned char* vbase = static_cast<const unsigned char*>(a.v) + plane;
+  const int ipt = kTileKeys / IK;
+  const int ntiles = (nmine + ipt - 1) / ipt;
+
+  auto issue = [&](int t) {  // warp 0
+    const int slot = t % kStages;
+    const int f = t * ipt, cnt = min(ipt, nmine - f);
+    int bytes = 0;
+    for (int x = lane; x < cnt; x += 32) bytes += item_at(f + x).y * kRowB;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], static_cast<uint32_t>(2 * bytes));
+    __syncwarp();
+    for (int x = lane; x < cnt; x += 32) {
+      const int2 e = item_at(f + x);
+      if (e.y > 0) {
+        const size_t src = static_cast<size_t>(e.x) * kRowB;
+        const uint32_t nb = static_cast<uint32_t>(e.y * kRowB);
+        bulk_g2s(kring + slot * kTileBytes + x * IK * kRowB, kbase + src, nb, &bars[slot]);
+        bulk_g2s(vring + slot * kTileBytes + x * IK * kRowB, vbase + src, nb, &bars[slot]);
+      }
+    }
+  };
+
+  float acc[RC][16];
+#pragma unroll
+  for (int r = 0; r < RC; ++r)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[r][e] = 0.0f;
+  float m_run = -INFINITY, l_run = 0.0f;  // valid in warp r for row r
+  bool timed_out = false;
+
+  if (warp == 0)
+    for (int t = 0; t < min(kStages - 1, ntiles); ++t) issue(t);
+
+  for (int t = 0; t < ntiles; ++t) {
+    if (warp == 0 && t + kStages - 1 < ntiles) issue(t + kStages - 1);
+    const int slot = t % kStages;
+    if (!mbar_wait(&bars[slot], (t / kStages) & 1)) timed_out = true;
+    const int f = t * ipt, cnt = min(ipt, nmine - f);
+    const unsigned char* ktile = kring + slot * kTileBytes;
+    const unsigned char* vtile = vring + slot * kTileBytes;
+
+    bool kvalid[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      const int kk = p * 32 + warp * 4 + grp;
+      const int item = kk / IK, kt = kk - item * IK;
+      int64_t j = -1;
+      if (item < cnt) {
+        const int2 e = item_at(f + item);
+        if (kt < e.y) j = static_cast<int64_t>(e.x) + kt;
+      }
+      kvalid[p] = j >= 0;
+      float kx[16];
+      load_row16<T>(ktile + kk * kRowB, lane8, kx);
+      float part[RC];
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        float x = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x = __fmaf_rn(qreg[r][e], kx[e], x);
+        part[r] = x;
+      }
+      const float dot = group_reduce_rows<RC>(part, lane8);
+      const int row = group_row_of_lane<RC>(lane8);
+      const bool ok = j >= 0 && row < R && j <= q_first + row % nrows;
+      if ((lane8 & ((8 / RC) - 1)) == 0) s_sm[row * kTileKeys + kk] = ok ? dot * a.scale_log2 : -INFINITY;
+    }
+    __syncthreads();
+    // online softmax, one warp per row
+    if (warp < RC) {
+      const int r = warp;
+      float sv[kPasses];
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int p = 0; p < kPasses; ++p) {
+        sv[p] = s_sm[r * kTileKeys + p * 32 + lane];
+        tmax = fmaxf(tmax, sv[p]);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+      const float m_new = fmaxf(m_run, tmax);
+      const float alpha = m_new == -INFINITY ? 1.0f : exp2f(m_run - m_new);
+      float psum = 0.0f;
+#pragma unroll
+      for (int p = 0; p < kPasses; ++p) {
+        const float pv = sv[p] == -INFINITY ? 0.0f : exp2f(sv[p] - m_new);
+        p_sm[(p * 32 + lane) * RC + r] = pv;
+        psum += pv;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+      l_run = l_run * alpha + psum;
+      m_run = m_new;
+      if (lane == 0) alpha_sm[r] = alpha;
+    }
+    __syncthreads();
+    float al[RC];
+#pragma unroll
+    for (int r = 0; r < RC; ++r) al[r] = alpha_sm[r];
+#pragma unroll
+    for (int r = 0; r < RC; ++r)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[r][e] *= al[r];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      if (!kvalid[p]) continue;
+      const int kk = p * 32 + warp * 4 + grp;
+      float vx[16];
+      load_row16<T>(vtile + kk * kRowB, lane8, vx);
+      float pk[RC];
+#pragma unroll
+      for (int r = 0; r < RC; ++r) pk[r] = p_sm[kk * RC + r];
+#pragma unroll
+      for (int r = 0; r < RC; ++r)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[r][e] = __fmaf_rn(pk[r], vx[e], acc[r][e]);
+    }
+    __syncthreads();
+  }
+
+  // ---- reduce the 4 key groups of a warp, then the 8 warps
+#pragma unroll
+  for (int r = 0; r < RC; ++r)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float x = acc[r][e];
+      x += __shfl_xor_sync(0xffffffffu, x, 8);
+      x += __shfl_xor_sync(0xffffffffu, x, 16);
+      acc[r][e] = x;
+    }
+  float* red = reinterpret_cast<float*>(kring);  // ring is idle now: [warp][RC][128]
+  if (grp == 0) {
+#pragma unroll
+    for (int r = 0; r < RC; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        red[(warp * RC + r) * kD + lane8 * 8 + e] = acc[r][e];
+        red[(warp * RC + r) * kD + 64 + lane8 * 8 + e] = acc[r][8 + e];
+      }
+  }
+  if (warp < RC && lane == 0) {
+    ml_sm[2 * warp] = m_run;
+    ml_sm[2 * warp + 1] = l_run;
+  }
+  __syncthreads();
+  for (int x = tid; x < R * kD; x += kThreads) {
+    const int r = x / kD, e = x % kD;
+    float o = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) o += red[(w * RC + r) * kD + e];
+    const int h = g * a.group + r / nrows, i = i0 + r % nrows;
+    const int64_t grow = (static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i;
+    const float m = ml_sm[2 * r], l = ml_sm[2 * r + 1];
+    if (a.nsplit == 1) {
+      const float val = l > 0.0f ? o / l : 0.0f;
+      if (sizeof(T) == 2)
+        reinterpret_cast<uint16_t*>(a.out)[grow * kD + e] = f2bf16_rn(val);
+      else
+        reinterpret_cast<float*>(a.out)[grow * kD + e] = val;
+    } else {
+      float* pr = a.part + (grow * a.nsplit + split) * (kD + 2);
+      if (e == 0) {
+        pr[0] = m;
+        pr[1] = l;
+      }
+      pr[2 + e] = o;
+    }
+  }
+  if (timed_out) report(a.status, kStatusTimeout, 2);
+}
+
+// Merge the splits of every query row: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+template <typename T>
+__global__ void __launch_bounds__(kD) attn_combine_kernel(const float* part, void* out, int nsplit) {
+  const int64_t row = blockIdx.x;
+  const int e = threadIdx.x;
+  const float* pr = part + row * nsplit * (kD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * (kD + 2)]);
+  float l = 0.0f, o = 0.0f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float ms = pr[s * (kD + 2)];
+      if (ms == -INFINITY) continue;
+      const float w = exp2f(ms - M);
+      l = __fmaf_rn(w, pr[s * (kD + 2) + 1], l);
+      o = __fmaf_rn(w, pr[s * (kD + 2) + 2 + e], o);
+    }
+  }
+  const float val = l > 0.0f ? o / l : 0.0f;
+  if (sizeof(T) == 2)
+    reinterpret_cast<uint16_t*>(out)[row * kD + e] = f2bf16_rn(val);
+  else
+    reinterpret_cast<float*>(out)[row * kD + e] = val;
+}
+
+template <typename T, int RC>
+cudaError_t launch_attn_t(const AttnArgs& a, int smem, cudaStream_t stream) {
+  auto kern = attn_fma_kernel<T, RC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nsplit, a.nqb * a.n_kvheads, a.batch);
+  kern<<<grid, kThreads, smem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.nsplit == 1) return e;
+  attn_combine_kernel<T><<<static_cast<unsigned>(a.rows_total), kD, 0, stream>>>(a.part, a.out,
+                                                                                 a.nsplit);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_attn_rc(const AttnArgs& a, int smem, cudaStream_t s) {
+  const int R = a.rows_max;
+  if (R <= 1) return launch_attn_t<T, 1>(a, smem, s);
+  if (R <= 2) return launch_attn_t<T, 2>(a, smem, s);
+  if (R <= 4) return launch_attn_t<T, 4>(a, smem, s);
+  return launch_attn_t<T, 8>(a, smem, s);
+}
+
+}  // namespace
+
+int attn_fma_tile_keys(int dtype) { return kTileBytes / (dtype == 1 ? 256 : 512); }
+
+int attn_fma_smem_bytes(int dtype, int rows_max, int table_items) {
+  const int rc = rows_max <= 1 ? 1 : rows_max <= 2 ? 2 : rows_max <= 4 ? 4 : 8;
+  return attn_smem_layout(attn_fma_tile_keys(dtype), rc, table_items).total;
+}
+
+cudaError_t launch_attn_fma(const AttnArgs& a, int smem, cudaStream_t stream) {
+  return a.dtype == 1 ? launch_attn_rc<uint16_t>(a, smem, stream)
+                      : launch_attn_rc<float>(a, smem, stream);
+}
+
+}  // namespace hips

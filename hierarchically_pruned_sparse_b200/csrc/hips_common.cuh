@@ -1,0 +1,209 @@
+// Device helpers shared by the hierarchically pruned attention kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hips {
+
+constexpr int kD = 128;            // head_dim
+constexpr int kThreads = 256;      // threads of the CUDA-core kernels
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxN0 = 2048;       // topk / block_k
+constexpr unsigned kStatusTimeout = 1u;
+constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
+
+// Status block at the head of every workspace (sticky error bits).
+struct Status {
+  unsigned int flags;
+  unsigned int where;
+};
+
+__device__ __forceinline__ void report(Status* st, unsigned bits, unsigned where) {
+  if (st) {
+    atomicOr(&st->flags, bits);
+    atomicExch(&st->where, where);
+  }
+}
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity; gives up after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+
+// Bulk (non-tensor) async copy global -> this CTA's shared memory, completing
+// on an mbarrier. dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------- numbers
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint16_t f2bf16_rn(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7f800000u) == 0x7f800000u) return static_cast<uint16_t>((u >> 16) | ((u & 0xffff) ? 0x40 : 0));
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+// Order-preserving map of a float score onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t score_key(float f) {
+  if (f == 0.0f) f = 0.0f;  // -0 and +0 are the same score
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Load the 16 elements a lane owns in the canonical order (slices lane and
+// lane + 8 of 8 consecutive elements each) of one 128-element row.
+template <typename T>
+__device__ __forceinline__ void load_row16(const unsigned char* row, int lane8, float (&x)[16]);
+
+template <>
+__device__ __forceinline__ void load_row16<uint16_t>(const unsigned char* row, int lane8,
+                                                     float (&x)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(row + lane8 * 16);
+  const uint4 b = *reinterpret_cast<const uint4*>(row + 128 + lane8 * 16);
+  x[0] = bf16lo(a.x); x[1] = bf16hi(a.x); x[2] = bf16lo(a.y); x[3] = bf16hi(a.y);
+  x[4] = bf16lo(a.z); x[5] = bf16hi(a.z); x[6] = bf16lo(a.w); x[7] = bf16hi(a.w);
+  x[8] = bf16lo(b.x); x[9] = bf16hi(b.x); x[10] = bf16lo(b.y); x[11] = bf16hi(b.y);
+  x[12] = bf16lo(b.z); x[13] = bf16hi(b.z); x[14] = bf16lo(b.w); x[15] = bf16hi(b.w);
+}
+
+template <>
+__device__ __forceinline__ void load_row16<float>(const unsigned char* row, int lane8,
+                                                  float (&x)[16]) {
+  const float4* p0 = reinterpret_cast<const float4*>(row + lane8 * 32);
+  const float4* p1 = reinterpret_cast<const float4*>(row + 256 + lane8 * 32);
+  const float4 a = p0[0], b = p0[1], c = p1[0], d = p1[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  x[8] = c.x; x[9] = c.y; x[10] = c.z; x[11] = c.w; x[12] = d.x; x[13] = d.y; x[14] = d.z;
+  x[15] = d.w;
+}
+
+template <typename T>
+constexpr int row_bytes() { return kD * static_cast<int>(sizeof(T)); }
+
+// Canonical-order reduction of RC lane partials over the 8 lanes of a group:
+// level 1 adds lanes (l, l^4), level 2 (l, l^2), level 3 (l, l^1), i.e.
+// ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7)) for every dot. With RC = 2^r dots a
+// lane keeps half of its dots at each of the first r levels, so afterwards
+// lane l holds dot (l >> (3 - r)) (the same sum tree, fewer shuffles).
+template <int RC>
+__device__ __forceinline__ float group_reduce_rows(float (&v)[RC], int lane8) {
+  static_assert(RC == 1 || RC == 2 || RC == 4 || RC == 8, "RC");
+#pragma unroll
+  for (int level = 0; level < 3; ++level) {
+    const int off = 4 >> level;
+    const int have = (RC >> level) > 1 ? (RC >> level) : 1;  // dots still held
+    if (have > 1) {
+      const int half = have / 2;
+      const bool upper = (lane8 & off) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? v[i] : v[i + half];
+        const float keep = upper ? v[i + half] : v[i];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+        v[i] = keep + recv;
+      }
+    } else {
+      v[0] = v[0] + __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+  return v[0];
+}
+
+template <int RC>
+__device__ __forceinline__ int group_row_of_lane(int lane8) {
+  return RC == 8 ? lane8 : RC == 4 ? (lane8 >> 1) : RC == 2 ? (lane8 >> 2) : 0;
+}
+
+// Exclusive block-wide prefix sum over kThreads threads; `total` gets the sum.
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int& total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < kWarps ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kWarps) scratch[lane] = t;
+  }
+  __syncthreads();
+  const int before = w ? scratch[w - 1] : 0;
+  total = scratch[kWarps - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+__device__ __forceinline__ int block_max_int(int v, int* scratch) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) scratch[w] = v;
+  __syncthreads();
+  int r = scratch[0];
+#pragma unroll
+  for (int i = 1; i < kWarps; ++i) r = max(r, scratch[i]);
+  __syncthreads();
+  return r;
+}
+
+}  // namespace hips

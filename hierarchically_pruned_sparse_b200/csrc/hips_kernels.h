@@ -1,0 +1,46 @@
+// Launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hips {
+
+struct Status;
+
+struct MaskArgs {
+  const void* q;
+  const void* k;
+  int32_t* idx;
+  Status* status;
+  int dtype, n_qheads, n_kvheads, group, q_len, block_q, block_k, n0max, sink, window;
+  int nqb, cluster, per_cta, rows_max, rows_pad;
+  int64_t units, seq_len, kv_cap, q_pos0, row_stride;
+};
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* idx;
+  void* out;
+  float* part;  // split partials [rows_total][nsplit][2 + 128]
+  Status* status;
+  int dtype, batch, n_qheads, n_kvheads, group, q_len, block_q, nqb, nsplit, dense, rows_max;
+  int item_keys, table_items;
+  int64_t rows_total, seq_len, mask_len, kv_cap, q_pos0, row_stride;
+  float scale_log2;
+};
+
+// CUDA-core hierarchical top-k mask (mask_fma.cu)
+int mask_fma_rc(int rows_max);
+int mask_fma_smem_bytes(int n0max, int rows_pad, int per_cta);
+int mask_fma_tile_keys(int dtype);
+cudaError_t launch_mask_fma(const MaskArgs& a, int smem, cudaStream_t stream);
+
+// CUDA-core split-K attention + combine (attn_fma.cu)
+int attn_fma_tile_keys(int dtype);
+int attn_fma_smem_bytes(int dtype, int rows_max, int table_items);
+cudaError_t launch_attn_fma(const AttnArgs& a, int smem, cudaStream_t stream);
+
+}  // namespace hips

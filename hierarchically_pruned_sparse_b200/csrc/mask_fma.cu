@@ -1,0 +1,442 @@
+// Hierarchical top-k mask on CUDA cores (decode and small query blocks).
+//
+// Method: "A Training-free Sub-quadratic Cost Transformer Model Serving
+// Framework With Hierarchically Pruned Attention", Author Rebuttal to the
+// Reviewer RsGC, Q2, steps 1-4: n0 = min(k/b_k, N) chunks tile the block range
+// [0, N) of the causal keys; every round halves each chunk, scores each half
+// by its centre block (max over the group's query rows and the block's keys
+// of q.k) and keeps the global top n0 halves; the loop stops when every chunk
+// is a single block. The kept blocks are then merged with the always-kept
+// sink and sliding-window blocks (research-map summary, "Add V 2k and D 1k")
+// into one ascending idx row with its nnz (Author Rebuttal to the Reviewer
+// NLBm, W2).
+//
+// Design (one launch for all rounds):
+//  * one thread-block cluster of C CTAs per mask row (sequence, KV head,
+//    query block); the candidates of a round are split over the C CTAs;
+//  * representative key blocks are gathered into a 3-stage shared-memory ring
+//    with bulk async copies (cp.async.bulk, completing on mbarriers);
+//  * each selection dot is evaluated in fp32 in one fixed order (8 lanes x 16
+//    elements, fma chains, then the tree ((p0+p4)+(p2+p6))+((p1+p5)+(p3+p7)))
+//    so the integer decision (which halves survive) is reproducible;
+//  * the C CTAs exchange their candidate scores through distributed shared
+//    memory; every CTA then runs the same radix select for the n0-th largest
+//    (score desc, position asc) key and the same order-preserving compaction,
+//    so all CTAs hold the identical chunk list (kept in ascending order, which
+//    makes the final kept set sorted without a sort);
+//  * CTA 0 writes the idx row: sink blocks, kept blocks between sink and
+//    window, window blocks.
+#include <cooperative_groups.h>
+
+#include "hips_common.cuh"
+#include "hips_kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace hips {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kTileBytes = 32768;
+
+struct MaskSmem {
+  int ring, bars, qs, chunk_s, chunk_e, cand_s, cand_e, keys, scores, key_max, hist, scratch,
+      total;
+};
+
+__host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline MaskSmem mask_smem_layout(int n0max, int rows_pad, int per_cta) {
+  MaskSmem L;
+  int o = 0;
+  L.ring = o;      o += kStages * kTileBytes;
+  L.bars = o;      o += align_up(kStages * 8, 16);
+  L.qs = o;        o += rows_pad * kD * 4;
+  L.chunk_s = o;   o += align_up(n0max * 4, 16);
+  L.chunk_e = o;   o += align_up(n0max * 4, 16);
+  L.cand_s = o;    o += align_up(2 * n0max * 4, 16);
+  L.cand_e = o;    o += align_up(2 * n0max * 4, 16);
+  L.keys = o;      o += align_up(2 * n0max * 4, 16);
+  L.scores = o;    o += align_up(2 * per_cta * 4, 16);
+  L.key_max = o;   o += 128 * 4;
+  L.hist = o;      o += 256 * 4;
+  L.scratch = o;   o += 64 * 4;
+  L.total = o;
+  return L;
+}
+
+// n-th largest key (1-based `want`) among keys[0, n); on return `want` is its
+// rank among the keys equal to it.
+__device__ uint32_t radix_select_desc(const uint32_t* keys, int n, int& want, int* hist,
+                                      int* bcast) {
+  uint32_t prefix = 0, pmask = 0;
+  const int lane = threadIdx.x & 31;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const uint32_t u = keys[i];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      int c[8], s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[255 - 8 * lane - j];
+        s += c[j];
+      }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - s;
+      if (excl < want && want <= incl) {
+        int acc = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (acc < want && want <= acc + c[j]) {
+            bcast[0] = 255 - 8 * lane - j;
+            bcast[1] = want - acc;
+          }
+          acc += c[j];
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t digit = static_cast<uint32_t>(bcast[0]);
+    want = bcast[1];
+    prefix |= digit << shift;
+    pmask |= 0xffu << shift;
+  }
+  return prefix;
+}
+
+template <typename T, int RC>
+__global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane8 = lane & 7, grp = lane >> 3;
+
+  const int64_t unit = blockIdx.y;
+  const int qb = static_cast<int>(unit % a.nqb);
+  const int g = static_cast<int>((unit / a.nqb) % a.n_kvheads);
+  const int b = static_cast<int>(unit / (static_cast<int64_t>(a.nqb) * a.n_kvheads));
+  const int i0 = qb * a.block_q;
+  const int nrows = min(a.block_q, a.q_len - i0);
+  const int R = a.group * nrows;
+  const int64_t q_first = a.q_pos0 + i0, q_last = q_first + nrows - 1;
+  const int64_t Tc = min(q_last + 1, a.seq_len);
+  const int bk = a.block_k;
+  const int64_t N = (Tc + bk - 1) / bk;
+  const int n0 = static_cast<int>(min64(a.n0max, N));
+  const int per_cta = a.per_cta;
+
+  const MaskSmem L = mask_smem_layout(a.n0max, a.rows_pad, per_cta);
+  unsigned char* ring = smem + L.ring;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  float* qs = reinterpret_cast<float*>(smem + L.qs);
+  int* chunk_s = reinterpret_cast<int*>(smem + L.chunk_s);
+  int* chunk_e = reinterpret_cast<int*>(smem + L.chunk_e);
+  int* cand_s = reinterpret_cast<int*>(smem + L.cand_s);
+  int* cand_e = reinterpret_cast<int*>(smem + L.cand_e);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
+  float* scores = reinterpret_cast<float*>(smem + L.scores);
+  float* key_max = reinterpret_cast<float*>(smem + L.key_max);
+  int* hist = reinterpret_cast<int*>(smem + L.hist);
+  int* scratch = reinterpret_cast<int*>(smem + L.scratch);
+  Status* status = a.status;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  // query rows of the group in fp32: row r = (head h, query i) -> h * nrows + i
+  const unsigned char* qbytes = static_cast<const unsigned char*>(a.q);
+  for (int e = tid; e < a.rows_pad * kD; e += kThreads) {
+    const int r = e / kD, c = e % kD;
+    float x = 0.0f;
+    if (r < R) {
+      const int h = g * a.group + r / nrows, i = i0 + r % nrows;
+      const int64_t off = ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i) * kD + c;
+      if (sizeof(T) == 2)
+        x = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(qbytes)[off]) << 16);
+      else
+        x = reinterpret_cast<const float*>(qbytes)[off];
+    }
+    qs[e] = x;
+  }
+  // step 1: n0 chunks that tile [0, N)
+  for (int i = tid; i < n0; i += kThreads) {
+    chunk_s[i] = static_cast<int>(static_cast<int64_t>(i) * N / n0);
+    chunk_e[i] = static_cast<int>(static_cast<int64_t>(i + 1) * N / n0);
+  }
+  __syncthreads();
+
+  const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
+                               (static_cast<int64_t>(b) * a.n_kvheads + g) * a.kv_cap * row_bytes<T>();
+  constexpr int kRowB = row_bytes<T>();
+  constexpr int kTileKeys = kTileBytes / kRowB;
+  constexpr int kPasses = kTileKeys / 32;
+  const int cpt = kTileKeys / bk;  // candidates per tile
+  const int nrc = a.rows_pad / RC;
+
+  float qreg[RC][16];
+  auto load_q = [&](int rc) {
+#pragma unroll
+    for (int r = 0; r < RC; ++r) {
+      const float* qr = qs + (rc * RC + r) * kD;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        qreg[r][e] = qr[lane8 * 8 + e];
+        qreg[r][8 + e] = qr[64 + lane8 * 8 + e];
+      }
+    }
+  };
+  if (nrc == 1) load_q(0);
+
+  uint32_t seq = 0;  // tiles consumed so far (ring position and phase)
+  int buf = 0;
+  bool timed_out = false;
+
+  for (;;) {
+    // ---- step 2: candidates (halves of every chunk; a 1-block chunk stays whole)
+    const int per_t = (n0 + kThreads - 1) / kThreads;
+    const int lo_t = min(n0, tid * per_t), hi_t = min(n0, lo_t + per_t);
+    int cnt = 0, longest = 0;
+    for (int i = lo_t; i < hi_t; ++i) {
+      const int len = chunk_e[i] - chunk_s[i];
+      cnt += len > 1 ? 2 : 1;
+      longest = max(longest, len);
+    }
+    longest = block_max_int(longest, scratch);
+    if (longest <= 1) break;
+    int ncand;
+    int pos = block_excl_scan(cnt, scratch, ncand);
+    for (int i = lo_t; i < hi_t; ++i) {
+      const int s = chunk_s[i], e = chunk_e[i], len = e - s;
+      if (len > 1) {
+        const int m = s + len / 2;
+        cand_s[pos] = s; cand_e[pos] = m; ++pos;
+        cand_s[pos] = m; cand_e[pos] = e; ++pos;
+      } else {
+        cand_s[pos] = s; cand_e[pos] = e; ++pos;
+      }
+    }
+    __syncthreads();
+
+    // ---- step 3: score this CTA's share of the candidates
+    const int c_lo = min(ncand, rank * per_cta), c_hi = min(ncand, c_lo + per_cta);
+    const int ntiles = (c_hi - c_lo + cpt - 1) / cpt;
+    float* my_scores = scores + buf * per_cta;
+
+    auto issue = [&](int t, uint32_t n) {  // warp 0 only
+      const int slot = static_cast<int>(n % kStages);
+      const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
+      unsigned char* dst = ring + slot * kTileBytes;
+      int bytes = 0;
+      for (int lc = lane; lc < cc; lc += 32) {
+        const int c = cf + lc;
+        const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
+        const int64_t nv = min64(bk, Tc - rep * bk);
+        bytes += static_cast<int>(nv) * kRowB;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], static_cast<uint32_t>(bytes));
+      __syncwarp();
+      for (int lc = lane; lc < cc; lc += 32) {
+        const int c = cf + lc;
+        const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
+        const int64_t nv = min64(bk, Tc - rep * bk);
+        bulk_g2s(dst + lc * bk * kRowB, kbase + rep * bk * kRowB,
+                 static_cast<uint32_t>(nv * kRowB), &bars[slot]);
+      }
+    };
+
+    if (warp == 0) {
+      for (int t = 0; t < min(kStages - 1, ntiles); ++t) issue(t, seq + t);
+    }
+    for (int t = 0; t < ntiles; ++t) {
+      const uint32_t n = seq + t;
+      if (warp == 0 && t + kStages - 1 < ntiles) issue(t + kStages - 1, n + kStages - 1);
+      const int slot = static_cast<int>(n % kStages);
+      if (!mbar_wait(&bars[slot], (n / kStages) & 1u)) timed_out = true;
+      const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
+      const int nkeys = cc * bk;
+      const unsigned char* tile = ring + slot * kTileBytes;
+
+      float kmax[kPasses];
+#pragma unroll
+      for (int p = 0; p < kPasses; ++p) kmax[p] = -INFINITY;
+      for (int rc = 0; rc < nrc; ++rc) {
+        if (nrc > 1) load_q(rc);
+#pragma unroll
+        for (int p = 0; p < kPasses; ++p) {
+          const int kk = p * 32 + warp * 4 + grp;
+          if (p * 32 + warp * 4 >= nkeys) break;  // warp-uniform
+          float kx[16];
+          load_row16<T>(tile + kk * kRowB, lane8, kx);
+          float part[RC];
+#pragma unroll
+          for (int r = 0; r < RC; ++r) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc = __fmaf_rn(qreg[r][e], kx[e], acc);
+            part[r] = acc;
+          }
+          const float dot = group_reduce_rows<RC>(part, lane8);
+          const int row = rc * RC + group_row_of_lane<RC>(lane8);
+          const int lc = kk / bk;
+          bool ok = kk < nkeys && row < R;
+          if (ok) {
+            const int c = cf + lc;
+            const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
+            const int64_t j = rep * bk + (kk - lc * bk);
+            ok = j < Tc && j <= q_first + row % nrows;
+          }
+          float v = ok ? dot : -INFINITY;
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          kmax[p] = fmaxf(kmax[p], v);
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < kPasses; ++p) {
+        const int kk = p * 32 + warp * 4 + grp;
+        if (lane8 == 0 && kk < nkeys) key_max[kk] = kmax[p];
+      }
+      __syncthreads();
+      for (int lc = tid; lc < cc; lc += kThreads) {
+        float s = -INFINITY;
+        for (int t2 = 0; t2 < bk; ++t2) s = fmaxf(s, key_max[lc * bk + t2]);
+        my_scores[cf - c_lo + lc] = s;
+      }
+      __syncthreads();
+    }
+    seq += static_cast<uint32_t>(ntiles);
+
+    // ---- exchange scores across the cluster
+    cluster.sync();
+    for (int i = tid; i < ncand; i += kThreads) {
+      const int peer = i / per_cta;
+      const float* src = peer == rank ? my_scores : cluster.map_shared_rank(my_scores, peer);
+      keys[i] = score_key(src[i - peer * per_cta]);
+    }
+    __syncthreads();
+
+    // ---- step 4: global top n0 by (score desc, start asc)
+    int want = n0;
+    const uint32_t theta = radix_select_desc(keys, ncand, want, hist, scratch + 32);
+    const int per_c = (ncand + kThreads - 1) / kThreads;
+    const int lo_c = min(ncand, tid * per_c), hi_c = min(ncand, lo_c + per_c);
+    int packed = 0;
+    for (int i = lo_c; i < hi_c; ++i)
+      packed += (keys[i] > theta ? 1 : 0) + (keys[i] == theta ? (1 << 16) : 0);
+    int tot;
+    int run = block_excl_scan(packed, scratch, tot);
+    for (int i = lo_c; i < hi_c; ++i) {
+      const int gt_before = run & 0xffff, eq_before = run >> 16;
+      const bool gt = keys[i] > theta, eq = keys[i] == theta;
+      if (gt || (eq && eq_before < want)) {
+        const int dst = gt_before + min(eq_before, want);
+        chunk_s[dst] = cand_s[i];
+        chunk_e[dst] = cand_e[i];
+      }
+      run += (gt ? 1 : 0) + (eq ? (1 << 16) : 0);
+    }
+    __syncthreads();
+    buf ^= 1;
+  }
+
+  // ---- union with sink and window blocks, write the idx row (CTA 0)
+  if (rank == 0) {
+    const int64_t ns = min64((a.sink + bk - 1) / bk, N);
+    const int64_t cut = a.window > 0 ? max64(0, q_first - a.window + 1) / bk : N;
+    const int64_t lead = min(ns, cut);
+    // kept blocks in [ns, cut): chunk_s is ascending
+    int lo = 0, hi = n0;
+    {
+      int l = 0, h = n0;
+      while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < ns) l = m + 1; else h = m; }
+      lo = l;
+      l = lo; h = n0;
+      while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < cut) l = m + 1; else h = m; }
+      hi = l;
+    }
+    const int64_t mid = hi > lo ? hi - lo : 0;
+    const int64_t tail = a.window > 0 ? N - cut : 0;
+    const int64_t nnz = lead + mid + tail;
+    int32_t* row = a.idx + unit * a.row_stride;
+    for (int64_t t = tid; t < a.row_stride; t += kThreads) {
+      int64_t val;
+      if (t == 0) val = nnz;
+      else {
+        const int64_t e = t - 1;
+        if (e < lead) val = e;
+        else if (e < lead + mid) val = chunk_s[lo + (e - lead)];
+        else if (e < nnz) val = cut + (e - lead - mid);
+        else val = -1;
+      }
+      row[t] = static_cast<int32_t>(val);
+    }
+  }
+  if (timed_out) report(status, kStatusTimeout, 1);
+  cluster.sync();  // peers may still read this CTA's scores
+}
+
+template <typename T, int RC>
+cudaError_t launch_mask_t(const MaskArgs& a, int smem, cudaStream_t stream) {
+  auto kern = mask_fma_kernel<T, RC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  if (a.cluster > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.cluster, static_cast<unsigned>(a.units), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <typename T>
+cudaError_t launch_mask_rc(const MaskArgs& a, int smem, cudaStream_t s) {
+  const int R = a.rows_max;
+  if (R <= 1) return launch_mask_t<T, 1>(a, smem, s);
+  if (R <= 2) return launch_mask_t<T, 2>(a, smem, s);
+  if (R <= 4) return launch_mask_t<T, 4>(a, smem, s);
+  return launch_mask_t<T, 8>(a, smem, s);
+}
+
+}  // namespace
+
+int mask_fma_rc(int rows_max) { return rows_max <= 1 ? 1 : rows_max <= 2 ? 2 : rows_max <= 4 ? 4 : 8; }
+
+int mask_fma_smem_bytes(int n0max, int rows_pad, int per_cta) {
+  return mask_smem_layout(n0max, rows_pad, per_cta).total;
+}
+
+int mask_fma_tile_keys(int dtype) { return kTileBytes / (dtype == 1 ? 256 : 512); }
+
+cudaError_t launch_mask_fma(const MaskArgs& a, int smem, cudaStream_t stream) {
+  return a.dtype == 1 ? launch_mask_rc<uint16_t>(a, smem, stream)
+                      : launch_mask_rc<float>(a, smem, stream);
+}
+
+}  // namespace hips

@@ -1,0 +1,143 @@
+/*
+ * hip_sparse.h -- C ABI of the B200 (sm_100a) hierarchically pruned attention
+ * library (libhip_sparse.so).
+ *
+ * The method (HiP, "A Training-Free Sub-quadratic Cost Transformer Model
+ * Serving Framework with Hierarchically Pruned Attention") has two steps on
+ * its hot path, and this library exposes each as one call:
+ *
+ *   hip_mask         hierarchical top-k selection of key blocks per query
+ *                    block: start from k/b_k chunks that tile the causal key
+ *                    range, repeatedly halve every chunk, score each half by
+ *                    its centre key block and keep the global top k/b_k halves
+ *                    until every chunk is one b_k block; then add the
+ *                    always-kept sink and sliding-window blocks and write the
+ *                    sorted block list with its nnz.
+ *                    (Author Rebuttal to the Reviewer RsGC, Q2, steps 1-4;
+ *                    research-map summary, Approach and the "Add V 2k and D 1k"
+ *                    row of Measured effects.)
+ *   hip_sparse_attn  exact softmax attention of every query row over only the
+ *                    keys of its selected blocks ("the block sparse attention
+ *                    kernel receives the non-zero entries' indices and the
+ *                    number of non-zero entries (nnz) for each row": Author
+ *                    Rebuttal to the Reviewer NLBm, W2), plus every key
+ *                    appended since the mask was computed when a mask is
+ *                    reused for r_m decode steps (summary, Limitations).
+ *   hip_dense_attn   exact causal attention over every key; a comparison
+ *                    point only (the pages compare against FlashAttention2).
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or keeps them. Calls are asynchronous on params->stream
+ *    (a cudaStream_t; NULL is the legacy default stream), allocate nothing,
+ *    and never synchronise the device.
+ *  - Layouts (row-major, element type = params->dtype):
+ *      q, out   [batch, n_qheads, q_len, head_dim]
+ *      k, v     [batch, n_kvheads, kv_capacity, head_dim]
+ *      idx      int32 [batch, n_kvheads, n_qblocks, row_stride] with
+ *               n_qblocks = ceil(q_len / block_q) and row_stride =
+ *               hip_idx_row_stride(params); entry 0 of a row is nnz, then nnz
+ *               ascending key-block ids, then -1 padding.
+ *    Query head h reads KV head h / (n_qheads / n_kvheads). Query row i sits
+ *    at absolute position q_pos0 + i and sees keys j <= q_pos0 + i.
+ *  - head_dim must be 128. k, v, q, out must be 16-byte aligned.
+ *  - Every call needs a workspace of at least hip_workspace_size(params, op)
+ *    bytes (256-byte aligned, caller-owned). Its first 256 bytes are a sticky
+ *    status block: kernels only ever set bits there. Clear it once after
+ *    allocating (hip_workspace_init) and read it with hip_check_status.
+ *  - Return value: HIPS_OK (0) or a negative HIPS_ERR_* code. Argument errors
+ *    are found on the host before anything is launched. HIPS_ERR_CUDA means
+ *    a launch failed; hip_last_cuda_error() gives the cudaError_t.
+ */
+#ifndef HIP_SPARSE_H_
+#define HIP_SPARSE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HIPS_API __attribute__((visibility("default")))
+#else
+#define HIPS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum hips_status {
+  HIPS_OK = 0,
+  HIPS_ERR_INVALID_ARG = -1, /* null pointer, bad shape, head ratio, topk % block_k ... */
+  HIPS_ERR_UNSUPPORTED = -2, /* head_dim != 128, dtype, a shape no kernel covers */
+  HIPS_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or too small */
+  HIPS_ERR_CUDA = -4,        /* a CUDA launch failed */
+  HIPS_ERR_TIMEOUT = -5      /* a bounded device wait expired (from hip_check_status) */
+};
+
+enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1 };
+
+enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2 };
+
+typedef struct hips_params {
+  int32_t batch;      /* sequences */
+  int32_t n_qheads;   /* query heads; a multiple of n_kvheads */
+  int32_t n_kvheads;  /* key/value heads (GQA groups) */
+  int32_t head_dim;   /* 128 */
+  int64_t seq_len;    /* keys present now: T_cur */
+  int64_t mask_len;   /* keys present when the mask was computed (== seq_len
+                         for a fresh mask; < seq_len when reusing it) */
+  int64_t kv_capacity;/* allocated length of the key axis, >= seq_len */
+  int32_t q_len;      /* query rows per sequence: 1 for decode, T for prefill */
+  int32_t dtype;      /* enum hips_dtype of q, k, v and out (accumulation is fp32) */
+  int64_t q_pos0;     /* absolute position of query row 0; q_pos0 + q_len <= seq_len */
+  int32_t block_q;    /* query rows sharing one mask (b_q) */
+  int32_t block_k;    /* keys per block (b_k), a power of two */
+  int32_t topk;       /* key budget k; a multiple of block_k, topk/block_k <= 2048 */
+  int32_t sink;       /* leading keys always kept (0 = none) */
+  int32_t window;     /* sliding-window keys always kept (0 = none) */
+  int32_t reserved;   /* must be 0 */
+  void* workspace;    /* device scratch, see hip_workspace_size */
+  size_t workspace_bytes;
+  void* stream;       /* cudaStream_t */
+} hips_params;
+
+/* Entries of one idx row: 1 (nnz) + the largest possible nnz. */
+HIPS_API int64_t hip_idx_row_stride(const hips_params* params);
+
+/* Workspace bytes needed by one call of `op` (enum hips_op) with these
+ * params; 0 if the params are invalid. */
+HIPS_API size_t hip_workspace_size(const hips_params* params, int op);
+
+/* Zero the status block of params->workspace (async on params->stream). */
+HIPS_API int hip_workspace_init(const hips_params* params);
+
+/* Synchronise params->stream, read and clear the status block. Returns
+ * HIPS_OK, or HIPS_ERR_TIMEOUT if some kernel gave up a bounded wait since
+ * the last check (its outputs are then undefined). */
+HIPS_API int hip_check_status(const hips_params* params);
+
+/* Hierarchical top-k mask (see above). q: [B, Hq, q_len, d]; k: [B, Hkv,
+ * kv_capacity, d]; keys [0, seq_len) are visible. idx_out: int32 [B, Hkv,
+ * n_qblocks, row_stride], fully written (padding included). */
+HIPS_API int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* idx_out);
+
+/* Block-sparse attention over idx (as written by hip_mask at mask_len keys)
+ * plus the keys [mask_len, seq_len). out: [B, Hq, q_len, d] in dtype. */
+HIPS_API int hip_sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx,
+                    const hips_params* params, void* out);
+
+/* Dense causal attention over keys [0, seq_len); block/topk fields ignored. */
+HIPS_API int hip_dense_attn(const void* q, const void* k, const void* v, const hips_params* params,
+                   void* out);
+
+/* cudaError_t of the last failed launch on this thread (0 if none). */
+HIPS_API int hip_last_cuda_error(void);
+
+/* Static string for a hips_status code. */
+HIPS_API const char* hip_error_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HIP_SPARSE_H_ */

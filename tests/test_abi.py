@@ -1,0 +1,108 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/hip_sparse.h, and rejects bad arguments on the host
+before anything is launched (no compute call is made here)."""
+import os
+import re
+
+import pytest
+
+from hierarchically_pruned_sparse_b200 import binding as hb
+from hierarchically_pruned_sparse_b200 import build as hbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    hbuild.build()
+    return hb.load()
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"HIPS_API\s+[\w\s\*]+?\b(hip_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert len(declared) >= 9
+    assert set(hb.EXPORTS) <= set(declared)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_error_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert hb.error_string(code)
+    assert hb.error_string(-99) == "unknown status"
+
+
+def _decode_params(**kw):
+    base = dict(batch=1, n_qheads=32, n_kvheads=8, seq_len=131072, q_len=1, q_pos0=131071,
+                dtype=hb.HIPS_BF16, block_q=1, block_k=2, topk=2048, sink=128, window=1024)
+    base.update(kw)
+    return hb.params(**base)
+
+
+def test_row_stride_and_workspace_sizes():
+    p = _decode_params()
+    # 1 (nnz) + topk/bk + ceil(sink/bk) + ceil((window + bq - 1)/bk) + 1
+    assert hb.idx_row_stride(p) == 1 + 1024 + 64 + 512 + 1
+    assert hb.workspace_size(p, hb.OP_MASK) >= 256
+    assert hb.workspace_size(p, hb.OP_SPARSE) > 256  # split-K partials
+    assert hb.workspace_size(p, hb.OP_DENSE) > 256
+    p2 = _decode_params(window=0, sink=0)
+    assert hb.idx_row_stride(p2) == 1 + 1024
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(n_qheads=30), hb.HIPS_ERR_INVALID_ARG),        # head ratio
+    (dict(topk=2047), hb.HIPS_ERR_INVALID_ARG),          # topk % block_k
+    (dict(block_k=3, topk=3 * 512), hb.HIPS_ERR_INVALID_ARG),  # block_k not a power of two
+    (dict(head_dim=64), hb.HIPS_ERR_UNSUPPORTED),
+    (dict(dtype=7), hb.HIPS_ERR_UNSUPPORTED),
+    (dict(q_pos0=131072), hb.HIPS_ERR_INVALID_ARG),      # query past the cache
+    (dict(mask_len=131073), hb.HIPS_ERR_INVALID_ARG),
+    (dict(kv_capacity=1000), hb.HIPS_ERR_INVALID_ARG),
+    (dict(topk=2 * 4096), hb.HIPS_ERR_UNSUPPORTED),      # more than 2048 chunks
+    (dict(batch=0), hb.HIPS_ERR_INVALID_ARG),
+    (dict(sink=-1), hb.HIPS_ERR_INVALID_ARG),
+])
+def test_bad_arguments_rejected_on_host(bad, code):
+    p = _decode_params(**bad)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    assert hb.mask_ptr(fake, fake, p, fake) == code
+    assert hb.sparse_attn_ptr(fake, fake, fake, fake, p, fake) == code
+    assert hb.workspace_size(p, hb.OP_MASK) == 0
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = _decode_params(workspace=1 << 20, workspace_bytes=1 << 30)
+    f = 1 << 20
+    assert hb.mask_ptr(0, f, p, f) == hb.HIPS_ERR_INVALID_ARG
+    assert hb.mask_ptr(f, 0, p, f) == hb.HIPS_ERR_INVALID_ARG
+    assert hb.mask_ptr(f, f, p, 0) == hb.HIPS_ERR_INVALID_ARG
+    assert hb.mask_ptr(f + 8, f, p, f) == hb.HIPS_ERR_INVALID_ARG  # q not 16-byte aligned
+    assert hb.sparse_attn_ptr(f, f, f, 0, p, f) == hb.HIPS_ERR_INVALID_ARG
+    assert hb.dense_attn_ptr(f, f, 0, p, f) == hb.HIPS_ERR_INVALID_ARG
+
+
+def test_workspace_checked_before_launch():
+    f = 1 << 20
+    p = _decode_params()  # no workspace
+    assert hb.mask_ptr(f, f, p, f) == hb.HIPS_ERR_WORKSPACE
+    need = hb.workspace_size(p, hb.OP_SPARSE)
+    p = _decode_params(workspace=f, workspace_bytes=need - 1)
+    assert hb.sparse_attn_ptr(f, f, f, f, p, f) == hb.HIPS_ERR_WORKSPACE
+    p = _decode_params(workspace=f + 16, workspace_bytes=need)  # not 256-byte aligned
+    assert hb.sparse_attn_ptr(f, f, f, f, p, f) == hb.HIPS_ERR_WORKSPACE
+
+
+def test_prefill_shapes_plan():
+    p = hb.params(batch=1, n_qheads=32, n_kvheads=8, seq_len=32768, q_len=32768, q_pos0=0,
+                  dtype=hb.HIPS_BF16, block_q=64, block_k=2, topk=2048, sink=128, window=1024)
+    assert hb.idx_row_stride(p) == 1 + 1024 + 64 + 544 + 1

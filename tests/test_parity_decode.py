@@ -1,0 +1,163 @@
+"""GPU parity of the decode path (and small query blocks) against the oracle.
+
+Masks must match the oracle bit-exactly except in rows whose oracle cut gap
+is below 1e-3 (q.k/sqrt(d) units), which must stay under 0.5% of rows.
+Attention is checked twice: fed the oracle's idx (isolates the attention
+kernel) and end to end from the CUDA mask.
+"""
+import functools
+
+import numpy as np
+import pytest
+
+import oracle
+from hierarchically_pruned_sparse_b200 import workloads as W
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    import torch
+    from hierarchically_pruned_sparse_b200 import build
+    assert torch.cuda.is_available(), "gpu tests need a CUDA device"
+    build.build()
+    oracle.set_threads(0)
+
+
+@functools.lru_cache(maxsize=4)
+def _inputs(w: W.Workload):
+    return W.make_inputs(w)
+
+
+def _session(bkw):
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    return hb.Session(**bkw)
+
+
+def _run_step(w, step=0, idx_ref=None):
+    """Returns (gpu idx, oracle idx, gap, gpu out e2e, gpu out on oracle idx, oracle out)."""
+    import torch
+    x = _inputs(w)
+    osh, bkw = pu.shapes(w, step)
+    q, k, v = pu.torch_inputs(x, w, step)
+    s = _session(bkw)
+    # the mask of a refresh is computed at mask_len keys
+    s.set(seq_len=w.seq_len, q_pos0=osh.q_pos0 - step)
+    q0 = pu.torch_inputs(x, w, 0)[0]
+    idx_g = s.mask(q0, k)
+    s.set(seq_len=osh.seq_len, q_pos0=osh.q_pos0)
+    osh0, _ = pu.shapes(w, 0)
+    osh0.kv_capacity = w.capacity
+    if idx_ref is None:
+        idx_ref, gap, _ = oracle.mask(x["q"][0], x["k"], osh0)
+    else:
+        idx_ref, gap = idx_ref
+    out_e2e = s.sparse_attn(q, k, v, idx_g)
+    idx_ref_dev = torch.from_numpy(idx_ref).to("cuda").reshape(idx_g.shape).contiguous()
+    out_on_ref = s.sparse_attn(q, k, v, idx_ref_dev)
+    torch.cuda.synchronize()
+    s.check()
+    out_ref = oracle.attention(x["q"][step], x["k"], x["v"], idx_ref, osh)
+    return (idx_g.cpu().numpy().reshape(idx_ref.shape), idx_ref, gap,
+            out_e2e.float().cpu().numpy().reshape(out_ref.shape),
+            out_on_ref.float().cpu().numpy().reshape(out_ref.shape), out_ref)
+
+
+def _check(w, step=0):
+    idx_g, idx_ref, gap, out_e2e, out_on_ref, out_ref = _run_step(w, step)
+    st = pu.compare_masks(idx_g, idx_ref, gap)
+    pu.compare_outputs(out_on_ref, out_ref, w.dtype)
+    if st["mismatched"] == 0:
+        pu.compare_outputs(out_e2e, out_ref, w.dtype)
+    return st
+
+
+SMALL = [
+    # several tiles, ragged T (not a multiple of b_k), sink + window, GQA
+    W.Workload("r1", "decode", 1, 4, 1, 128, 5001, 1, 2, 256, 16, 100, "bf16", 4, "uniform"),
+    W.Workload("r2", "decode", 2, 8, 2, 128, 3001, 1, 4, 128, 0, 0, "bf16", 2, "uniform"),
+    W.Workload("r3", "decode", 1, 2, 2, 128, 777, 1, 1, 64, 3, 5, "f32", 2, "uniform"),
+    # N/n0 not a power of two: chunks of 11 and 12 blocks, single-block chunks pass through
+    W.Workload("r4", "decode", 1, 4, 1, 128, 3000, 1, 2, 256, 0, 0, "bf16", 2, "uniform"),
+    # budget >= T: every block kept (dense)
+    W.Workload("r5", "decode", 1, 4, 2, 128, 500, 1, 2, 512, 0, 0, "bf16"),
+    # 8 query heads per KV head
+    W.Workload("r6", "decode", 1, 8, 1, 128, 4096, 1, 2, 512, 32, 64, "bf16", 4, "uniform"),
+    # one key per block, long
+    W.Workload("r7", "decode", 1, 1, 1, 128, 20000, 1, 1, 1024, 0, 0, "f32", 4, "uniform"),
+    # 16-key blocks in bf16, 2 query heads per group
+    W.Workload("r8", "decode", 1, 4, 2, 128, 9000, 1, 16, 1024, 64, 256, "bf16", 4, "uniform"),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_decode(w):
+    _check(w)
+
+
+def test_decode_8k_f32():
+    st = _check(W.DECODE_8K_F32)
+    assert st["mismatched"] == 0
+
+
+def test_decode_128k_llama_shape():
+    _check(W.DECODE_128K)
+
+
+def test_dense_attention_128k():
+    import torch
+    w = W.DECODE_128K
+    x = _inputs(w)
+    osh, bkw = pu.shapes(w)
+    q, k, v = pu.torch_inputs(x, w)
+    s = _session(bkw)
+    out = s.dense_attn(q, k, v)
+    torch.cuda.synchronize()
+    s.check()
+    ref = oracle.attention(x["q"][0], x["k"], x["v"], None, osh)
+    pu.compare_outputs(out.float().cpu().numpy().reshape(ref.shape), ref, w.dtype)
+
+
+def test_small_prefill_blocks_on_cuda_cores():
+    # query blocks of 4 rows x 2 heads: the CUDA-core mask and attention kernels
+    import torch
+    w = W.Workload("p1", "prefill", 1, 4, 2, 128, 700, 4, 2, 128, 8, 16, "bf16")
+    x = _inputs(w)
+    osh, bkw = pu.shapes(w)
+    q, k, v = pu.torch_inputs(x, w)
+    s = _session(bkw)
+    idx = s.mask(q, k)
+    out = s.sparse_attn(q, k, v, idx)
+    torch.cuda.synchronize()
+    s.check()
+    idx_ref, gap, _ = oracle.mask(x["q"][0], x["k"], osh)
+    st = pu.compare_masks(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref, gap)
+    ref = oracle.attention(x["q"][0], x["k"], x["v"], idx_ref, osh)
+    if st["mismatched"] == 0:
+        pu.compare_outputs(out.float().cpu().numpy().reshape(ref.shape), ref, w.dtype)
+
+
+def test_mask_reuse_small():
+    w = W.Workload("m1", "decode", 2, 4, 1, 128, 3000, 1, 2, 256, 16, 64, "bf16", 2,
+                   "uniform", refresh=5)
+    for step in range(w.refresh):
+        _check(w, step)
+
+
+def test_batched_decode_mask_reuse_128k():
+    w = W.DECODE_B16_REUSE
+    x = _inputs(w)
+    osh0, _ = pu.shapes(w, 0)
+    idx_ref, gap, _ = oracle.mask(x["q"][0], x["k"], osh0)
+    for step in (0, 3, 7):
+        idx_g, _, _, out_e2e, out_on_ref, out_ref = _run_step(w, step, (idx_ref, gap))
+        st = pu.compare_masks(idx_g, idx_ref, gap)
+        pu.compare_outputs(out_on_ref, out_ref, w.dtype)
+        if st["mismatched"] == 0:
+            pu.compare_outputs(out_e2e, out_ref, w.dtype)
+
+
+def test_decode_1m():
+    _check(W.DECODE_1M)
