@@ -344,8 +344,16 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(const float* part, voi
 template <typename T, int RC>
 cudaError_t launch_attn_t(const AttnArgs& a, int smem, cudaStream_t stream) {
   auto kern = attn_fma_kernel<T, RC>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static int smem_set[kMaxDevices] = {};  // once per kernel and device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  dev %= kMaxDevices;
+  if (smem > smem_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = smem;
+  }
   dim3 grid(a.nsplit, a.nqb * a.n_kvheads, a.batch);
   kern<<<grid, kThreads, smem, stream>>>(a);
   e = cudaGetLastError();

@@ -10,6 +10,7 @@ constexpr int kD = 128;            // head_dim
 constexpr int kThreads = 256;      // threads of the CUDA-core kernels
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxN0 = 2048;       // topk / block_k
+constexpr int kMaxDevices = 64;
 constexpr unsigned kStatusTimeout = 1u;
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 

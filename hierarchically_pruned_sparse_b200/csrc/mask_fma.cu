@@ -394,11 +394,22 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
 template <typename T, int RC>
 cudaError_t launch_mask_t(const MaskArgs& a, int smem, cudaStream_t stream) {
   auto kern = mask_fma_kernel<T, RC>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // attributes are set once per kernel (not inside a later stream capture)
+  static int smem_set[kMaxDevices] = {};
+  static bool big_cluster_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (a.cluster > 8) {
+  dev %= kMaxDevices;
+  if (smem > smem_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = smem;
+  }
+  if (a.cluster > 8 && !big_cluster_set[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
+    big_cluster_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.cluster, static_cast<unsigned>(a.units), 1);
