@@ -16,6 +16,8 @@ HIPS_ERR_UNSUPPORTED = -2
 HIPS_ERR_WORKSPACE = -3
 HIPS_ERR_CUDA = -4
 HIPS_ERR_TIMEOUT = -5
+HIPS_ERR_TOO_LARGE = -6
+NOALLOC_SCRATCH_BYTES = 1 << 20
 
 HIPS_F32 = 0
 HIPS_BF16 = 1
@@ -81,6 +83,8 @@ def load() -> ctypes.CDLL:
     lib.hip_sparse_attn.argtypes = [vp, vp, vp, vp, P, vp]
     lib.hip_dense_attn.restype = ctypes.c_int
     lib.hip_dense_attn.argtypes = [vp, vp, vp, P, vp]
+    lib.hip_sparse_attn_noalloc.restype = ctypes.c_int
+    lib.hip_sparse_attn_noalloc.argtypes = [vp, vp, vp, vp, P, vp]
     lib.hip_last_cuda_error.restype = ctypes.c_int
     lib.hip_last_cuda_error.argtypes = []
     lib.hip_error_string.restype = ctypes.c_char_p
@@ -137,6 +141,12 @@ def sparse_attn_ptr(q: int, k: int, v: int, idx: int, p: Params, out: int) -> in
                                       ctypes.byref(p), out or None))
 
 
+def sparse_attn_noalloc_ptr(q: int, k: int, v: int, idx: int, p: Params, out: int) -> int:
+    """hip_sparse_attn on the library's fixed scratch array (no workspace)."""
+    return int(load().hip_sparse_attn_noalloc(q or None, k or None, v or None, idx or None,
+                                              ctypes.byref(p), out or None))
+
+
 def dense_attn_ptr(q: int, k: int, v: int, p: Params, out: int) -> int:
     return int(load().hip_dense_attn(q or None, k or None, v or None, ctypes.byref(p),
                                      out or None))
@@ -167,6 +177,13 @@ def hip_mask(q, k, p: Params, idx_out) -> None:
 
 def hip_sparse_attn(q, k, v, idx, p: Params, out) -> None:
     _check("hip_sparse_attn", sparse_attn_ptr(_dev(q), _dev(k), _dev(v), _dev(idx), p, _dev(out)))
+
+
+def hip_sparse_attn_noalloc(q, k, v, idx, p: Params, out) -> None:
+    """Sparse attention for callers that cannot allocate device memory: the
+    split-K scratch is a fixed array inside the library (see the header)."""
+    _check("hip_sparse_attn_noalloc",
+           sparse_attn_noalloc_ptr(_dev(q), _dev(k), _dev(v), _dev(idx), p, _dev(out)))
 
 
 def hip_dense_attn(q, k, v, p: Params, out) -> None:

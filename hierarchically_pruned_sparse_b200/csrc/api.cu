@@ -188,6 +188,33 @@ int run_attention(const void* q, const void* k, const void* v, const int32_t* id
 
 }  // namespace
 
+namespace hips {
+
+// Validation and launch plan of a sparse attention call that brings its own
+// scratch memory (no caller workspace); *scratch_bytes is what it needs.
+int plan_sparse_attn_own_scratch(const void* q, const void* k, const void* v, const int32_t* idx,
+                                 const hips_params* p, void* out, AttnArgs* args, int* smem,
+                                 size_t* scratch_bytes) {
+  int st = validate(p, HIPS_OP_SPARSE);
+  if (st) return st;
+  if (!q || !k || !v || !out || !idx) return HIPS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(idx, 4))
+    return HIPS_ERR_INVALID_ARG;
+  AttnPlan plan;
+  st = plan_attn(p, false, &plan);
+  if (st) return st;
+  *args = plan.a;
+  args->q = q; args->k = k; args->v = v; args->idx = idx; args->out = out;
+  *smem = plan.smem;
+  *scratch_bytes = plan.ws;
+  return HIPS_OK;
+}
+
+int record_cuda_error(cudaError_t e) { return cuda_status(e); }
+
+}  // namespace hips
+
 extern "C" {
 
 int64_t hip_idx_row_stride(const hips_params* params) {
@@ -279,6 +306,7 @@ const char* hip_error_string(int status) {
     case HIPS_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case HIPS_ERR_CUDA: return "CUDA launch failed";
     case HIPS_ERR_TIMEOUT: return "a bounded device wait expired";
+    case HIPS_ERR_TOO_LARGE: return "request exceeds the library's built-in scratch size";
     default: return "unknown status";
   }
 }

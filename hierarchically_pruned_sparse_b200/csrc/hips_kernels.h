@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+struct hips_params;
+
 namespace hips {
 
 struct Status;
@@ -42,5 +44,12 @@ cudaError_t launch_mask_fma(const MaskArgs& a, int smem, cudaStream_t stream);
 int attn_fma_tile_keys(int dtype);
 int attn_fma_smem_bytes(int dtype, int rows_max, int table_items);
 cudaError_t launch_attn_fma(const AttnArgs& a, int smem, cudaStream_t stream);
+
+// Plan of a sparse attention call that uses scratch memory of its own
+// (api.cu); the no-allocation entry point in noalloc.cu launches it.
+int plan_sparse_attn_own_scratch(const void* q, const void* k, const void* v, const int32_t* idx,
+                                 const hips_params* p, void* out, AttnArgs* args, int* smem,
+                                 size_t* scratch_bytes);
+int record_cuda_error(cudaError_t e);
 
 }  // namespace hips

@@ -71,7 +71,8 @@ enum hips_status {
   HIPS_ERR_UNSUPPORTED = -2, /* head_dim != 128, dtype, a shape no kernel covers */
   HIPS_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or too small */
   HIPS_ERR_CUDA = -4,        /* a CUDA launch failed */
-  HIPS_ERR_TIMEOUT = -5      /* a bounded device wait expired (from hip_check_status) */
+  HIPS_ERR_TIMEOUT = -5,     /* a bounded device wait expired (from hip_check_status) */
+  HIPS_ERR_TOO_LARGE = -6    /* more scratch than hip_sparse_attn_noalloc's fixed array */
 };
 
 enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1 };
@@ -129,6 +130,31 @@ HIPS_API int hip_sparse_attn(const void* q, const void* k, const void* v, const 
 /* Dense causal attention over keys [0, seq_len); block/topk fields ignored. */
 HIPS_API int hip_dense_attn(const void* q, const void* k, const void* v, const hips_params* params,
                    void* out);
+
+/* Same result as hip_sparse_attn, for callers that cannot allocate device
+ * memory: for example a serving loop whose memory pool is frozen after
+ * start-up, or code that must not let a cudaMalloc (and the device-wide
+ * synchronisation it may imply) into a latency-critical decode step. It takes
+ * no workspace (params->workspace and workspace_bytes are ignored) and calls
+ * no allocator; its split-K scratch is a fixed device array of
+ * HIPS_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits. There is no counterpart to this
+ * call in the paper; it only changes where the scratch lives.
+ *  - Calls needing more scratch than that (hip_workspace_size(params,
+ *    HIPS_OP_SPARSE) > HIPS_NOALLOC_SCRATCH_BYTES) return HIPS_ERR_TOO_LARGE
+ *    before launching anything.
+ *  - The first call on each device looks the array's device address up
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; each call clears the part that must start at zero. Calls that
+ *    overlap on the GPU (different streams, or other host threads) race on
+ *    it: serialise them.
+ *  - Bounded-wait failures of this call are not reported through
+ *    hip_check_status (it has no caller workspace). */
+#define HIPS_NOALLOC_SCRATCH_BYTES (1u << 20)
+HIPS_API int hip_sparse_attn_noalloc(const void* q, const void* k, const void* v,
+                                     const int32_t* idx, const hips_params* params, void* out);
 
 /* cudaError_t of the last failed launch on this thread (0 if none). */
 HIPS_API int hip_last_cuda_error(void);
