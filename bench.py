@@ -410,7 +410,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     mask_gbs = mask_bytes / (mask_ms * 1e-3) / 1e9
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
     step_gbs = (mask_bytes + attn_bytes) / (total_ms * 1e-3 / (steps)) / 1e9
-    nsplit_launches = 3 if hb.workspace_size(sess.p, hb.OP_SPARSE) > 256 else 2
+    launches_per_step = 2  # hip_mask + hip_sparse_attn (the split merge is fused)
 
     # e2e: per step, H2D of the step's query and new key/value rows from pinned
     # host memory, the two C-ABI calls, D2H of the output; captured as a graph
@@ -478,7 +478,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         "kernels": {"how": "CUDA event nodes around each call, last full graph replay of the timed region",
                     "mask_us": mask_ms * 1e3, "mask_bytes": mask_bytes, "mask_gbs": mask_gbs,
                     "attn_us": attn_ms * 1e3, "attn_bytes": attn_bytes, "attn_gbs": attn_gbs},
-        "gpu_launches": nsplit_launches * steps,
+        "gpu_launches": launches_per_step * steps,
         "clocks": clk.summary(),
     }
     if e2e:

@@ -17,7 +17,7 @@ HIPS_ERR_WORKSPACE = -3
 HIPS_ERR_CUDA = -4
 HIPS_ERR_TIMEOUT = -5
 HIPS_ERR_TOO_LARGE = -6
-NOALLOC_SCRATCH_BYTES = 1 << 20
+NOALLOC_SCRATCH_BYTES = 512 << 10
 
 HIPS_F32 = 0
 HIPS_BF16 = 1

@@ -15,7 +15,12 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kPlanSMs = 148;         // B200 streaming multiprocessors
-constexpr size_t kStatusBytes = 256;  // head of every workspace
+// Head of every workspace: bytes [0, 256) hold the sticky status word, bytes
+// [256, 4096) one split-merge counter per (sequence, KV head, query block)
+// unit of a split attention call; both are zero between calls.
+constexpr size_t kStatusBytes = 4096;
+constexpr size_t kCounterOffset = 256;
+constexpr int64_t kMaxCounters = (kStatusBytes - kCounterOffset) / 4;
 constexpr int kMaxSmem = 227 * 1024;
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -61,7 +66,29 @@ struct MaskPlan {
   hips::MaskArgs a;
   int smem;
   size_t ws;
+  bool mma;  // tensor-core kernel (bf16) or CUDA-core kernel
 };
+
+// Tensor-core mask plan: bf16, up to 256 query rows per mask, b_k <= 32.
+int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
+  hips::MaskArgs& a = plan->a;
+  const int nc = hips::mask_mma_nc(a.rows_max);
+  if (p->dtype != HIPS_BF16 || nc == 0 || p->block_k > 32 || a.units > 65535)
+    return HIPS_ERR_UNSUPPORTED;
+  const int cpt = hips::mask_mma_tile_keys() / p->block_k;
+  const int64_t ncand = 2 * static_cast<int64_t>(a.n0max);
+  int c = 1;
+  while (c < cluster_cap && a.units * (2 * c) <= kPlanSMs && cdiv(ncand, 2 * c) >= cpt) c *= 2;
+  a.cluster = c;
+  a.per_cta = static_cast<int>(cdiv(ncand, c));
+  a.rows_pad = nc * 16;
+  a.stages = 0;
+  plan->smem = hips::mask_mma_smem_bytes(nc, a.n0max, a.per_cta, c);
+  if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
+  plan->mma = true;
+  plan->ws = kStatusBytes;
+  return HIPS_OK;
+}
 
 int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   hips::MaskArgs& a = plan->a;
@@ -83,6 +110,8 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   a.q_pos0 = p->q_pos0;
   a.row_stride = row_stride(p);
   a.rows_max = group_rows(p, p->block_q);
+  plan->mma = false;
+  if (plan_mask_mma(p, cluster_cap, plan) == HIPS_OK) return HIPS_OK;
   if (a.rows_max > 32 || a.units > 65535) return HIPS_ERR_UNSUPPORTED;
   const int rc = hips::mask_fma_rc(a.rows_max);
   a.rows_pad = static_cast<int>(cdiv(a.rows_max, rc) * rc);
@@ -94,10 +123,37 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   while (c < cluster_cap && a.units * (2 * c) <= kPlanSMs && cdiv(ncand, 2 * c) >= cpt) c *= 2;
   a.cluster = c;
   a.per_cta = static_cast<int>(cdiv(ncand, c));
-  plan->smem = hips::mask_fma_smem_bytes(a.n0max, a.rows_pad, a.per_cta);
+  a.stages = 3;
+  plan->smem = hips::mask_fma_smem_bytes(a.n0max, a.rows_pad, a.per_cta, c, a.stages);
+  if (plan->smem > kMaxSmem) {
+    a.stages = 2;
+    plan->smem = hips::mask_fma_smem_bytes(a.n0max, a.rows_pad, a.per_cta, c, a.stages);
+  }
   if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
   plan->ws = kStatusBytes;
   return HIPS_OK;
+}
+
+// Clusters of this plan's shape that fit on the device at once, cached per
+// device and shape (queried once, outside any stream capture in practice).
+int resident_clusters(const MaskPlan& plan) {
+  struct Entry { int dev, dtype, rows, cluster, smem, n; };
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const hips::MaskArgs& a = plan.a;
+  const int rows = plan.mma ? 100 + hips::mask_mma_nc(a.rows_max) : hips::mask_fma_rc(a.rows_max);
+  for (int i = 0; i < used; ++i) {
+    const Entry& e = cache[i];
+    if (e.dev == dev && e.dtype == a.dtype && e.rows == rows && e.cluster == a.cluster &&
+        e.smem == plan.smem)
+      return e.n;
+  }
+  const int n = plan.mma ? hips::mask_mma_max_active_clusters(a, plan.smem)
+                         : hips::mask_fma_max_active_clusters(a, plan.smem);
+  if (used < 64) cache[used++] = Entry{dev, a.dtype, rows, a.cluster, plan.smem, n};
+  return n;
 }
 
 // ---------------------------------------------------------------- attention plan
@@ -142,14 +198,16 @@ int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
     w_max = (a.row_stride - 1) + cdiv(std::max<int64_t>(0, p->seq_len - p->mask_len), a.item_keys);
   }
   const int64_t units = static_cast<int64_t>(p->batch) * p->n_kvheads * a.nqb;
-  int64_t nsplit = std::min<int64_t>(cdiv(2 * kPlanSMs, units), cdiv(w_max, ipt));
-  nsplit = std::max<int64_t>(1, std::min<int64_t>(nsplit, 1024));
+  // one wave: splits x units <= SMs (one CTA per SM), at least a tile per split
+  int64_t nsplit = std::min<int64_t>(kPlanSMs / units, cdiv(w_max, ipt));
+  nsplit = std::max<int64_t>(1, nsplit);
+  if (nsplit > 1 && units > kMaxCounters) nsplit = 1;
   a.nsplit = static_cast<int>(nsplit);
   a.table_items = dense ? 0 : static_cast<int>(cdiv(w_max, nsplit));
   plan->smem = hips::attn_fma_smem_bytes(p->dtype, a.rows_max, a.table_items);
   if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
   size_t part = 0;
-  if (a.nsplit > 1) part = static_cast<size_t>(a.rows_total) * a.nsplit * (hips::kD + 2) * sizeof(float);
+  if (a.nsplit > 1) part = static_cast<size_t>(a.rows_total) * a.nsplit * (hips::kD + 4) * sizeof(float);
   plan->ws = kStatusBytes + (part + 255) / 256 * 256;
   return HIPS_OK;
 }
@@ -183,6 +241,7 @@ int run_attention(const void* q, const void* k, const void* v, const int32_t* id
   a.q = q; a.k = k; a.v = v; a.idx = idx; a.out = out;
   a.status = static_cast<hips::Status*>(p->workspace);
   a.part = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + kStatusBytes);
+  a.counters = reinterpret_cast<unsigned int*>(static_cast<char*>(p->workspace) + kCounterOffset);
   return cuda_status(hips::launch_attn_fma(a, plan.smem, static_cast<cudaStream_t>(p->stream)));
 }
 
@@ -266,16 +325,22 @@ int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* i
   st = check_workspace(params, plan.ws);
   if (st) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
-  // A 16-CTA cluster needs 16 free SMs of one GPC; fall back to smaller
-  // clusters if the device refuses the shape.
+  // A cluster of C CTAs needs C free SMs of one GPC. Take the largest cluster
+  // for which every mask row is resident at once (one wave); fall back to
+  // smaller clusters if the device refuses the shape.
   for (int cap = 16; cap >= 1; cap /= 2) {
     st = plan_mask(params, cap, &plan);
     if (st) return st;
     if (plan.a.cluster > cap) continue;
+    if (plan.a.cluster > 1 && cap > 1) {
+      const int fit = resident_clusters(plan);
+      if (fit >= 0 && fit < plan.a.units) continue;
+    }
     hips::MaskArgs& a = plan.a;
     a.q = q; a.k = k; a.idx = idx_out;
     a.status = static_cast<hips::Status*>(params->workspace);
-    const cudaError_t e = hips::launch_mask_fma(a, plan.smem, stream);
+    const cudaError_t e = plan.mma ? hips::launch_mask_mma(a, plan.smem, stream)
+                                   : hips::launch_mask_fma(a, plan.smem, stream);
     if (e == cudaSuccess) return HIPS_OK;
     if ((e == cudaErrorInvalidClusterSize || e == cudaErrorLaunchOutOfResources) && cap > 1) {
       (void)cudaGetLastError();

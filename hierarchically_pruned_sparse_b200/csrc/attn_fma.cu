@@ -11,11 +11,16 @@
 //
 // Design: grid (splits, KV head x query block, sequence). A split takes a
 // contiguous range of work items (one key block each); K and V rows of a
-// 64-key tile are gathered with bulk async copies into a 3-stage ring, the
+// 64-key tile are gathered by all threads with 16-byte cp.async copies into a
+// 3-stage ring (completion tracked on one mbarrier per stage), the
 // G query heads of the group share every gathered tile, and each of 8 warps
 // works on 4 keys at a time with 8 lanes per key (16 head elements per lane).
 // Scores go through an fp32 online softmax (exp2 domain); each split writes
-// (m, l, unnormalised o) and the combine kernel merges the splits.
+// (m, l, unnormalised o) to the workspace and the last split of a unit to
+// finish (an atomic ticket; nobody waits) merges them into the output. The
+// grid is one wave (splits x units <= SM count). The kernel is launched with
+// programmatic stream serialisation: everything before the grid-dependency
+// wait (barrier set-up, query loads) overlaps the tail of the mask kernel.
 #include "hips_common.cuh"
 #include "hips_kernels.h"
 
@@ -25,6 +30,7 @@ namespace {
 
 constexpr int kStages = 3;
 constexpr int kTileBytes = 16384;  // one of K or V per stage
+constexpr int kPartStride = kD + 4; // m, l, pad, pad, o[128]: o 16-byte aligned
 
 struct AttnSmem {
   int kring, vring, bars, table, s, p, alpha, ml, total;
@@ -42,7 +48,7 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int tile_keys, int rc, int 
   L.s = o;      o += align16(rc * tile_keys * 4);
   L.p = o;      o += align16(rc * tile_keys * 4);
   L.alpha = o;  o += align16(rc * 4);
-  L.ml = o;     o += align16(2 * rc * 4);
+  L.ml = o;     o += align16((2 * rc + 4) * 4);  // m, l per row; merge flag
   L.total = o;
   return L;
 }
@@ -76,6 +82,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   float* alpha_sm = reinterpret_cast<float*>(smem + L.alpha);
   float* ml_sm = reinterpret_cast<float*>(smem + L.ml);
 
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], kThreads);
+    fence_mbar_init();
+  }
+  // query rows in registers: lane holds 16 elements of each of the RC rows
+  float qreg[RC][16];
+  {
+    const T* qp = static_cast<const T*>(a.q);
+#pragma unroll
+    for (int r = 0; r < RC; ++r) {
+      if (r < R) {
+        const int h = g * a.group + r / nrows, i = i0 + r % nrows;
+        const unsigned char* row = reinterpret_cast<const unsigned char*>(
+            qp + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i) * kD);
+        load_row16<T>(row, lane8, qreg[r]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) qreg[r][e] = 0.0f;
+      }
+    }
+  }
+  // the idx rows may come from the kernel launched just before this one
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // ---- work items of this unit and this split's range
   const int64_t unit = (static_cast<int64_t>(b) * a.n_kvheads + g) * a.nqb + qb;
   const int32_t* idx_row = a.dense ? nullptr : a.idx + unit * a.row_stride;
@@ -93,10 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   const int64_t it_lo = min(nitems, split * per), it_hi = min(nitems, it_lo + per);
   const int nmine = static_cast<int>(it_hi - it_lo);
 
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-    fence_mbar_init();
-  }
   // item table (sparse): first key and key count of every item of this split;
   // ids read from idx are range-checked so a malformed row cannot drive reads
   // outside [0, seq_len)
@@ -123,48 +149,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   };
   __syncthreads();
 
-  // query rows in registers: lane holds 16 elements of each of the RC rows
-  float qreg[RC][16];
-  {
-    const T* qp = static_cast<const T*>(a.q);
-#pragma unroll
-    for (int r = 0; r < RC; ++r) {
-      if (r < R) {
-        const int h = g * a.group + r / nrows, i = i0 + r % nrows;
-        const unsigned char* row = reinterpret_cast<const unsigned char*>(
-            qp + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i) * kD);
-        load_row16<T>(row, lane8, qreg[r]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) qreg[r][e] = 0.0f;
-      }
-    }
-  }
-
   const size_t plane = (static_cast<size_t>(b) * a.n_kvheads + g) * static_cast<size_t>(a.kv_cap) * kRowB;
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) + plane;
   const unsigned char* vbase = static_cast<const unsigned char*>(a.v) + plane;
   const int ipt = kTileKeys / IK;
   const int ntiles = (nmine + ipt - 1) / ipt;
 
-  auto issue = [&](int t) {  // warp 0
+  constexpr int kChunks = kRowB / 16;  // 16-byte chunks per key row
+  auto issue = [&](int t) {  // all threads
     const int slot = t % kStages;
     const int f = t * ipt, cnt = min(ipt, nmine - f);
-    int bytes = 0;
-    for (int x = lane; x < cnt; x += 32) bytes += item_at(f + x).y * kRowB;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], static_cast<uint32_t>(2 * bytes));
-    __syncwarp();
-    for (int x = lane; x < cnt; x += 32) {
-      const int2 e = item_at(f + x);
-      if (e.y > 0) {
-        const size_t src = static_cast<size_t>(e.x) * kRowB;
-        const uint32_t nb = static_cast<uint32_t>(e.y * kRowB);
-        bulk_g2s(kring + slot * kTileBytes + x * IK * kRowB, kbase + src, nb, &bars[slot]);
-        bulk_g2s(vring + slot * kTileBytes + x * IK * kRowB, vbase + src, nb, &bars[slot]);
+    unsigned char* kd = kring + slot * kTileBytes;
+    unsigned char* vd = vring + slot * kTileBytes;
+    const int nchunks = cnt * IK * kChunks;
+    for (int i = tid; i < nchunks; i += kThreads) {
+      const int kk = i / kChunks, ch = i - kk * kChunks;
+      const int item = kk / IK, kt = kk - item * IK;
+      const int2 e = item_at(f + item);
+      if (kt < e.y) {
+        const size_t src = (static_cast<size_t>(e.x) + kt) * kRowB + ch * 16;
+        cp_async16(kd + kk * kRowB + ch * 16, kbase + src);
+        cp_async16(vd + kk * kRowB + ch * 16, vbase + src);
       }
     }
+    cp_async_arrive(&bars[slot]);
   };
 
   float acc[RC][16];
@@ -175,11 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   float m_run = -INFINITY, l_run = 0.0f;  // valid in warp r for row r
   bool timed_out = false;
 
-  if (warp == 0)
-    for (int t = 0; t < min(kStages - 1, ntiles); ++t) issue(t);
+  for (int t = 0; t < min(kStages - 1, ntiles); ++t) issue(t);
 
   for (int t = 0; t < ntiles; ++t) {
-    if (warp == 0 && t + kStages - 1 < ntiles) issue(t + kStages - 1);
+    if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
     const int slot = t % kStages;
     if (!mbar_wait(&bars[slot], (t / kStages) & 1)) timed_out = true;
     const int f = t * ipt, cnt = min(ipt, nmine - f);
@@ -305,40 +312,80 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
       else
         reinterpret_cast<float*>(a.out)[grow * kD + e] = val;
     } else {
-      float* pr = a.part + (grow * a.nsplit + split) * (kD + 2);
+      float* pr = a.part + (grow * a.nsplit + split) * kPartStride;
       if (e == 0) {
         pr[0] = m;
         pr[1] = l;
       }
-      pr[2 + e] = o;
+      pr[4 + e] = o;
     }
   }
   if (timed_out) report(a.status, kStatusTimeout, 2);
-}
+  if (a.nsplit == 1) return;
 
-// Merge the splits of every query row: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
-template <typename T>
-__global__ void __launch_bounds__(kD) attn_combine_kernel(const float* part, void* out, int nsplit) {
-  const int64_t row = blockIdx.x;
-  const int e = threadIdx.x;
-  const float* pr = part + row * nsplit * (kD + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * (kD + 2)]);
-  float l = 0.0f, o = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ms = pr[s * (kD + 2)];
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      l = __fmaf_rn(w, pr[s * (kD + 2) + 1], l);
-      o = __fmaf_rn(w, pr[s * (kD + 2) + 2 + e], o);
+  // ---- the last split of this unit to finish merges all splits:
+  // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
+  __threadfence();
+  __syncthreads();
+  int* flag = reinterpret_cast<int*>(ml_sm + 2 * RC);
+  if (tid == 0) *flag = atomicAdd(&a.counters[unit], 1u) == static_cast<unsigned>(a.nsplit - 1);
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  float* wts = reinterpret_cast<float*>(kring) + kWarps * RC * kD;  // [RC][nsplit]
+  float* lsum = ml_sm;                                              // [RC]
+  if (warp < R) {
+    const int r = warp;
+    const int h = g * a.group + r / nrows, i = i0 + r % nrows;
+    const int64_t grow = (static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i;
+    const float* base = a.part + grow * a.nsplit * kPartStride;
+    float M = -INFINITY;
+    for (int s = lane; s < a.nsplit; s += 32) M = fmaxf(M, __ldcg(base + s * kPartStride));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Ls = 0.0f;
+    for (int s = lane; s < a.nsplit; s += 32) {
+      const float ms = __ldcg(base + s * kPartStride);
+      const float w = (M == -INFINITY || ms == -INFINITY) ? 0.0f : exp2f(ms - M);
+      wts[r * a.nsplit + s] = w;
+      Ls = __fmaf_rn(w, __ldcg(base + s * kPartStride + 1), Ls);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    __syncwarp();
+    if (lane == 0) lsum[r] = Ls;
+  }
+  __syncthreads();
+  for (int x = tid; x < R * (kD / 4); x += kThreads) {
+    const int r = x / (kD / 4), d4 = (x % (kD / 4)) * 4;
+    const int h = g * a.group + r / nrows, i = i0 + r % nrows;
+    const int64_t grow = (static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + i;
+    const float* base = a.part + grow * a.nsplit * kPartStride + 4 + d4;
+    float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 8
+    for (int s = 0; s < a.nsplit; ++s) {
+      const float w = wts[r * a.nsplit + s];
+      const float4 ps = __ldcg(reinterpret_cast<const float4*>(base + s * kPartStride));
+      o.x = __fmaf_rn(w, ps.x, o.x);
+      o.y = __fmaf_rn(w, ps.y, o.y);
+      o.z = __fmaf_rn(w, ps.z, o.z);
+      o.w = __fmaf_rn(w, ps.w, o.w);
+    }
+    const float L = lsum[r];
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    const float v0 = o.x * inv, v1 = o.y * inv, v2 = o.z * inv, v3 = o.w * inv;
+    if (sizeof(T) == 2) {
+      uint16_t* dst = reinterpret_cast<uint16_t*>(a.out) + grow * kD + d4;
+      uint2 pk;
+      pk.x = static_cast<uint32_t>(f2bf16_rn(v0)) | (static_cast<uint32_t>(f2bf16_rn(v1)) << 16);
+      pk.y = static_cast<uint32_t>(f2bf16_rn(v2)) | (static_cast<uint32_t>(f2bf16_rn(v3)) << 16);
+      *reinterpret_cast<uint2*>(dst) = pk;
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + grow * kD + d4) =
+          make_float4(v0, v1, v2, v3);
     }
   }
-  const float val = l > 0.0f ? o / l : 0.0f;
-  if (sizeof(T) == 2)
-    reinterpret_cast<uint16_t*>(out)[row * kD + e] = f2bf16_rn(val);
-  else
-    reinterpret_cast<float*>(out)[row * kD + e] = val;
+  if (tid == 0) a.counters[unit] = 0;  // ready for the next call
 }
 
 template <typename T, int RC>
@@ -354,13 +401,17 @@ cudaError_t launch_attn_t(const AttnArgs& a, int smem, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     smem_set[dev] = smem;
   }
-  dim3 grid(a.nsplit, a.nqb * a.n_kvheads, a.batch);
-  kern<<<grid, kThreads, smem, stream>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || a.nsplit == 1) return e;
-  attn_combine_kernel<T><<<static_cast<unsigned>(a.rows_total), kD, 0, stream>>>(a.part, a.out,
-                                                                                 a.nsplit);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.nsplit, a.nqb * a.n_kvheads, a.batch);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <typename T>

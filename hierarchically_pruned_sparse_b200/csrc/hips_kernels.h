@@ -16,7 +16,7 @@ struct MaskArgs {
   int32_t* idx;
   Status* status;
   int dtype, n_qheads, n_kvheads, group, q_len, block_q, block_k, n0max, sink, window;
-  int nqb, cluster, per_cta, rows_max, rows_pad;
+  int nqb, cluster, per_cta, rows_max, rows_pad, stages;
   int64_t units, seq_len, kv_cap, q_pos0, row_stride;
 };
 
@@ -26,8 +26,9 @@ struct AttnArgs {
   const void* v;
   const int32_t* idx;
   void* out;
-  float* part;  // split partials [rows_total][nsplit][2 + 128]
+  float* part;  // split partials [rows_total][nsplit][4 + 128]
   Status* status;
+  unsigned int* counters;  // per unit, zero between calls (split merge tickets)
   int dtype, batch, n_qheads, n_kvheads, group, q_len, block_q, nqb, nsplit, dense, rows_max;
   int item_keys, table_items;
   int64_t rows_total, seq_len, mask_len, kv_cap, q_pos0, row_stride;
@@ -36,11 +37,20 @@ struct AttnArgs {
 
 // CUDA-core hierarchical top-k mask (mask_fma.cu)
 int mask_fma_rc(int rows_max);
-int mask_fma_smem_bytes(int n0max, int rows_pad, int per_cta);
+int mask_fma_smem_bytes(int n0max, int rows_pad, int per_cta, int cluster, int stages);
 int mask_fma_tile_keys(int dtype);
+// clusters of a.cluster CTAs that can be resident at once (-1 if unknown)
+int mask_fma_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_mask_fma(const MaskArgs& a, int smem, cudaStream_t stream);
 
-// CUDA-core split-K attention + combine (attn_fma.cu)
+// Tensor-core hierarchical top-k mask, bf16 (mask_mma.cu)
+int mask_mma_nc(int rows_max);  // N / 16 of the MMA (0 = too many rows)
+int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster);
+int mask_mma_tile_keys();
+int mask_mma_max_active_clusters(const MaskArgs& a, int smem);
+cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream);
+
+// CUDA-core split-K attention with the split merge fused (attn_fma.cu)
 int attn_fma_tile_keys(int dtype);
 int attn_fma_smem_bytes(int dtype, int rows_max, int table_items);
 cudaError_t launch_attn_fma(const AttnArgs& a, int smem, cudaStream_t stream);

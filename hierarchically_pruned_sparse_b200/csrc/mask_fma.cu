@@ -14,16 +14,21 @@
 // Design (one launch for all rounds):
 //  * one thread-block cluster of C CTAs per mask row (sequence, KV head,
 //    query block); the candidates of a round are split over the C CTAs;
-//  * representative key blocks are gathered into a 3-stage shared-memory ring
-//    with bulk async copies (cp.async.bulk, completing on mbarriers);
+//  * representative key blocks are gathered into a shared-memory ring by all
+//    threads with 16-byte cp.async copies (coalesced: 16 consecutive threads
+//    per key row), each stage completing on an mbarrier that every thread
+//    arrives on once its own copies land;
 //  * each selection dot is evaluated in fp32 in one fixed order (8 lanes x 16
 //    elements, fma chains, then the tree ((p0+p4)+(p2+p6))+((p1+p5)+(p3+p7)))
 //    so the integer decision (which halves survive) is reproducible;
 //  * the C CTAs exchange their candidate scores through distributed shared
-//    memory; every CTA then runs the same radix select for the n0-th largest
-//    (score desc, position asc) key and the same order-preserving compaction,
-//    so all CTAs hold the identical chunk list (kept in ascending order, which
-//    makes the final kept set sorted without a sort);
+//    memory; every CTA then runs the same selection, so all of them hold the
+//    identical chunk list. The selection is a bucket select: one histogram
+//    over 2048 buckets that are linear in the score between the round's min
+//    and max (monotone, so whole buckets are kept or dropped), then an exact
+//    rank by (score desc, start asc) among the members of the one bucket the
+//    cut falls in. Chunks stay in ascending order (order-preserving
+//    compaction), so the final kept set is sorted without a sort;
 //  * CTA 0 writes the idx row: sink blocks, kept blocks between sink and
 //    window, window blocks.
 #include <cooperative_groups.h>
@@ -37,91 +42,50 @@ namespace hips {
 
 namespace {
 
-constexpr int kStages = 3;
 constexpr int kTileBytes = 32768;
+constexpr int kBuckets = 2048;
+constexpr int kMaxPer = (2 * kMaxN0 + kThreads - 1) / kThreads;  // scores per thread
 
 struct MaskSmem {
-  int ring, bars, qs, chunk_s, chunk_e, cand_s, cand_e, keys, scores, key_max, hist, scratch,
-      total;
+  int ring, bars, qs, chunk_s, chunk_e, cand_s, cand_e, sc, bkt, keep, mem, scores, hist,
+      key_max, scratch, total;
 };
 
 __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline MaskSmem mask_smem_layout(int n0max, int rows_pad, int per_cta) {
+__host__ __device__ inline MaskSmem mask_smem_layout(int n0max, int rows_pad, int per_cta,
+                                                     int cluster, int stages) {
   MaskSmem L;
+  const int nc = 2 * n0max;
   int o = 0;
-  L.ring = o;      o += kStages * kTileBytes;
-  L.bars = o;      o += align_up(kStages * 8, 16);
+  L.ring = o;      o += stages * kTileBytes;
+  L.bars = o;      o += align_up(stages * 8, 16);
   L.qs = o;        o += rows_pad * kD * 4;
   L.chunk_s = o;   o += align_up(n0max * 4, 16);
   L.chunk_e = o;   o += align_up(n0max * 4, 16);
-  L.cand_s = o;    o += align_up(2 * n0max * 4, 16);
-  L.cand_e = o;    o += align_up(2 * n0max * 4, 16);
-  L.keys = o;      o += align_up(2 * n0max * 4, 16);
-  L.scores = o;    o += align_up(2 * per_cta * 4, 16);
+  L.cand_s = o;    o += align_up(nc * 4, 16);
+  L.cand_e = o;    o += align_up(nc * 4, 16);
+  L.sc = o;        o += align_up(nc * 4, 16);
+  L.bkt = o;       o += align_up(nc * 2, 16);
+  L.keep = o;      o += align_up(nc, 16);
+  L.mem = o;       o += align_up(nc * 4, 16);
+  L.scores = o;    o += cluster > 1 ? align_up(2 * per_cta * 4, 16) : 0;
+  L.hist = o;      o += kBuckets * 4;
   L.key_max = o;   o += 128 * 4;
-  L.hist = o;      o += 256 * 4;
   L.scratch = o;   o += 64 * 4;
   L.total = o;
   return L;
-}
-
-// n-th largest key (1-based `want`) among keys[0, n); on return `want` is its
-// rank among the keys equal to it.
-__device__ uint32_t radix_select_desc(const uint32_t* keys, int n, int& want, int* hist,
-                                      int* bcast) {
-  uint32_t prefix = 0, pmask = 0;
-  const int lane = threadIdx.x & 31;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-      const uint32_t u = keys[i];
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      int c[8], s = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = hist[255 - 8 * lane - j];
-        s += c[j];
-      }
-      int incl = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int excl = incl - s;
-      if (excl < want && want <= incl) {
-        int acc = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc < want && want <= acc + c[j]) {
-            bcast[0] = 255 - 8 * lane - j;
-            bcast[1] = want - acc;
-          }
-          acc += c[j];
-        }
-      }
-    }
-    __syncthreads();
-    const uint32_t digit = static_cast<uint32_t>(bcast[0]);
-    want = bcast[1];
-    prefix |= digit << shift;
-    pmask |= 0xffu << shift;
-  }
-  return prefix;
 }
 
 template <typename T, int RC>
 __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
+  const int C = a.cluster;
+  const int rank = C > 1 ? static_cast<int>(cluster.block_rank()) : 0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int lane8 = lane & 7, grp = lane >> 3;
+  const int stages = a.stages;
 
   const int64_t unit = blockIdx.y;
   const int qb = static_cast<int>(unit % a.nqb);
@@ -131,13 +95,13 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   const int nrows = min(a.block_q, a.q_len - i0);
   const int R = a.group * nrows;
   const int64_t q_first = a.q_pos0 + i0, q_last = q_first + nrows - 1;
-  const int64_t Tc = min(q_last + 1, a.seq_len);
+  const int64_t Tc = min64(q_last + 1, a.seq_len);
   const int bk = a.block_k;
   const int64_t N = (Tc + bk - 1) / bk;
   const int n0 = static_cast<int>(min64(a.n0max, N));
   const int per_cta = a.per_cta;
 
-  const MaskSmem L = mask_smem_layout(a.n0max, a.rows_pad, per_cta);
+  const MaskSmem L = mask_smem_layout(a.n0max, a.rows_pad, per_cta, C, stages);
   unsigned char* ring = smem + L.ring;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   float* qs = reinterpret_cast<float*>(smem + L.qs);
@@ -145,15 +109,17 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   int* chunk_e = reinterpret_cast<int*>(smem + L.chunk_e);
   int* cand_s = reinterpret_cast<int*>(smem + L.cand_s);
   int* cand_e = reinterpret_cast<int*>(smem + L.cand_e);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
-  float* scores = reinterpret_cast<float*>(smem + L.scores);
-  float* key_max = reinterpret_cast<float*>(smem + L.key_max);
+  float* sc = reinterpret_cast<float*>(smem + L.sc);
+  uint16_t* bkt = reinterpret_cast<uint16_t*>(smem + L.bkt);
+  uint8_t* keep = reinterpret_cast<uint8_t*>(smem + L.keep);
+  int* mem = reinterpret_cast<int*>(smem + L.mem);
+  float* scores = C > 1 ? reinterpret_cast<float*>(smem + L.scores) : sc;
   int* hist = reinterpret_cast<int*>(smem + L.hist);
+  float* key_max = reinterpret_cast<float*>(smem + L.key_max);
   int* scratch = reinterpret_cast<int*>(smem + L.scratch);
-  Status* status = a.status;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < stages; ++s) mbar_init(&bars[s], kThreads);
     fence_mbar_init();
   }
   // query rows of the group in fp32: row r = (head h, query i) -> h * nrows + i
@@ -176,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
     chunk_s[i] = static_cast<int>(static_cast<int64_t>(i) * N / n0);
     chunk_e[i] = static_cast<int>(static_cast<int64_t>(i + 1) * N / n0);
   }
+  for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
   __syncthreads();
 
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
@@ -185,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   constexpr int kPasses = kTileKeys / 32;
   const int cpt = kTileKeys / bk;  // candidates per tile
   const int nrc = a.rows_pad / RC;
+  const bool direct = bk <= 4;     // a candidate's keys sit in one warp pass
 
   float qreg[RC][16];
   auto load_q = [&](int rc) {
@@ -208,16 +176,17 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
     // ---- step 2: candidates (halves of every chunk; a 1-block chunk stays whole)
     const int per_t = (n0 + kThreads - 1) / kThreads;
     const int lo_t = min(n0, tid * per_t), hi_t = min(n0, lo_t + per_t);
-    int cnt = 0, longest = 0;
+    int cnt = 0, nlong = 0;
     for (int i = lo_t; i < hi_t; ++i) {
       const int len = chunk_e[i] - chunk_s[i];
       cnt += len > 1 ? 2 : 1;
-      longest = max(longest, len);
+      nlong += len > 1 ? 1 : 0;
     }
-    longest = block_max_int(longest, scratch);
-    if (longest <= 1) break;
-    int ncand;
-    int pos = block_excl_scan(cnt, scratch, ncand);
+    int tot;
+    int pos = block_excl_scan(cnt | (nlong << 16), scratch, tot);  // counts <= 4096 < 2^16
+    if ((tot >> 16) == 0) break;  // every chunk is one block: stop
+    const int ncand = tot & 0xffff;
+    pos &= 0xffff;
     for (int i = lo_t; i < hi_t; ++i) {
       const int s = chunk_s[i], e = chunk_e[i], len = e - s;
       if (len > 1) {
@@ -233,40 +202,31 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
     // ---- step 3: score this CTA's share of the candidates
     const int c_lo = min(ncand, rank * per_cta), c_hi = min(ncand, c_lo + per_cta);
     const int ntiles = (c_hi - c_lo + cpt - 1) / cpt;
-    float* my_scores = scores + buf * per_cta;
+    float* my_scores = scores + (C > 1 ? buf * per_cta : 0);
 
-    auto issue = [&](int t, uint32_t n) {  // warp 0 only
-      const int slot = static_cast<int>(n % kStages);
+    constexpr int kChunks = kRowB / 16;  // 16-byte chunks per key row
+    auto issue = [&](int t, uint32_t n) {  // all threads
+      const int slot = static_cast<int>(n % stages);
       const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
       unsigned char* dst = ring + slot * kTileBytes;
-      int bytes = 0;
-      for (int lc = lane; lc < cc; lc += 32) {
+      const int nchunks = cc * bk * kChunks;
+      for (int i = tid; i < nchunks; i += kThreads) {
+        const int kk = i / kChunks, ch = i - kk * kChunks;
+        const int lc = kk / bk;
         const int c = cf + lc;
         const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
-        const int64_t nv = min64(bk, Tc - rep * bk);
-        bytes += static_cast<int>(nv) * kRowB;
+        const int64_t j = rep * bk + (kk - lc * bk);
+        if (j < Tc) cp_async16(dst + kk * kRowB + ch * 16, kbase + j * kRowB + ch * 16);
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], static_cast<uint32_t>(bytes));
-      __syncwarp();
-      for (int lc = lane; lc < cc; lc += 32) {
-        const int c = cf + lc;
-        const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
-        const int64_t nv = min64(bk, Tc - rep * bk);
-        bulk_g2s(dst + lc * bk * kRowB, kbase + rep * bk * kRowB,
-                 static_cast<uint32_t>(nv * kRowB), &bars[slot]);
-      }
+      cp_async_arrive(&bars[slot]);
     };
 
-    if (warp == 0) {
-      for (int t = 0; t < min(kStages - 1, ntiles); ++t) issue(t, seq + t);
-    }
+    for (int t = 0; t < min(stages - 1, ntiles); ++t) issue(t, seq + t);
     for (int t = 0; t < ntiles; ++t) {
       const uint32_t n = seq + t;
-      if (warp == 0 && t + kStages - 1 < ntiles) issue(t + kStages - 1, n + kStages - 1);
-      const int slot = static_cast<int>(n % kStages);
-      if (!mbar_wait(&bars[slot], (n / kStages) & 1u)) timed_out = true;
+      if (t + stages - 1 < ntiles) issue(t + stages - 1, n + stages - 1);
+      const int slot = static_cast<int>(n % stages);
+      if (!mbar_wait(&bars[slot], (n / stages) & 1u)) timed_out = true;
       const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
       const int nkeys = cc * bk;
       const unsigned char* tile = ring + slot * kTileBytes;
@@ -276,10 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
       for (int p = 0; p < kPasses; ++p) kmax[p] = -INFINITY;
       for (int rc = 0; rc < nrc; ++rc) {
         if (nrc > 1) load_q(rc);
+        // all passes are computed (stale rows of a partial tile are masked
+        // below), so loads and fma chains of different passes can overlap
 #pragma unroll
         for (int p = 0; p < kPasses; ++p) {
           const int kk = p * 32 + warp * 4 + grp;
-          if (p * 32 + warp * 4 >= nkeys) break;  // warp-uniform
           float kx[16];
           load_row16<T>(tile + kk * kRowB, lane8, kx);
           float part[RC];
@@ -292,9 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
           }
           const float dot = group_reduce_rows<RC>(part, lane8);
           const int row = rc * RC + group_row_of_lane<RC>(lane8);
-          const int lc = kk / bk;
           bool ok = kk < nkeys && row < R;
           if (ok) {
+            const int lc = kk / bk;
             const int c = cf + lc;
             const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
             const int64_t j = rep * bk + (kk - lc * bk);
@@ -307,49 +268,160 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
           kmax[p] = fmaxf(kmax[p], v);
         }
       }
+      if (direct) {
+        // max over the b_k (<= 4) consecutive key groups of a candidate
 #pragma unroll
-      for (int p = 0; p < kPasses; ++p) {
-        const int kk = p * 32 + warp * 4 + grp;
-        if (lane8 == 0 && kk < nkeys) key_max[kk] = kmax[p];
-      }
-      __syncthreads();
-      for (int lc = tid; lc < cc; lc += kThreads) {
-        float s = -INFINITY;
-        for (int t2 = 0; t2 < bk; ++t2) s = fmaxf(s, key_max[lc * bk + t2]);
-        my_scores[cf - c_lo + lc] = s;
+        for (int p = 0; p < kPasses; ++p) {
+          float v = kmax[p];
+          if (bk >= 2) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          if (bk >= 4) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+          const int kk = p * 32 + warp * 4 + grp;
+          if (lane8 == 0 && (grp % bk) == 0 && kk < nkeys) my_scores[cf - c_lo + kk / bk] = v;
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < kPasses; ++p) {
+          const int kk = p * 32 + warp * 4 + grp;
+          if (lane8 == 0 && kk < nkeys) key_max[kk] = kmax[p];
+        }
+        __syncthreads();
+        for (int lc = tid; lc < cc; lc += kThreads) {
+          float s = -INFINITY;
+          for (int t2 = 0; t2 < bk; ++t2) s = fmaxf(s, key_max[lc * bk + t2]);
+          my_scores[cf - c_lo + lc] = s;
+        }
       }
       __syncthreads();
     }
     seq += static_cast<uint32_t>(ntiles);
 
-    // ---- exchange scores across the cluster
-    cluster.sync();
-    for (int i = tid; i < ncand; i += kThreads) {
-      const int peer = i / per_cta;
-      const float* src = peer == rank ? my_scores : cluster.map_shared_rank(my_scores, peer);
-      keys[i] = score_key(src[i - peer * per_cta]);
+    // ---- exchange scores across the cluster (batched DSMEM loads); track min/max
+    if (C > 1) cluster.sync();
+    float lo = INFINITY, hi = -INFINITY;
+    {
+      float v[kMaxPer];
+#pragma unroll
+      for (int j = 0; j < kMaxPer; ++j) {
+        const int i = tid + j * kThreads;
+        v[j] = 0.0f;
+        if (i < ncand) {
+          if (C > 1) {
+            const int peer = i / per_cta;
+            const float* src = cluster.map_shared_rank(my_scores, peer);
+            v[j] = src[i - peer * per_cta];
+          } else {
+            v[j] = sc[i];
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxPer; ++j) {
+        const int i = tid + j * kThreads;
+        if (i < ncand) {
+          float x = v[j];
+          if (x == 0.0f) x = 0.0f;  // -0 and +0 are the same score
+          sc[i] = x;
+          lo = fminf(lo, x);
+          hi = fmaxf(hi, x);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    float* red = reinterpret_cast<float*>(scratch + 16);  // 16 floats
+    if (lane == 0) {
+      red[warp] = lo;
+      red[8 + warp] = hi;
     }
     __syncthreads();
+    lo = red[0];
+    hi = red[8];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      lo = fminf(lo, red[w]);
+      hi = fmaxf(hi, red[8 + w]);
+    }
 
-    // ---- step 4: global top n0 by (score desc, start asc)
-    int want = n0;
-    const uint32_t theta = radix_select_desc(keys, ncand, want, hist, scratch + 32);
+    // ---- step 4: global top n0 by (score desc, start asc) -- bucket select
+    // bucket(s) = floor((s - lo) * scale) is non-decreasing in s, so a bucket
+    // above the cut bucket is kept whole and one below is dropped whole.
+    const float scale = hi > lo ? static_cast<float>(kBuckets - 1) / (hi - lo) : 0.0f;
+    for (int i = tid; i < ncand; i += kThreads) {
+      int bi = static_cast<int>((sc[i] - lo) * scale);
+      bi = min(max(bi, 0), kBuckets - 1);
+      bkt[i] = static_cast<uint16_t>(bi);
+      atomicAdd(&hist[bi], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns 64 buckets, lane 0 the top ones, scanned from the top
+      constexpr int kPerLane = kBuckets / 32;
+      const int top = kBuckets - kPerLane * lane;
+      int s = 0;
+      for (int j = 1; j <= kPerLane; ++j) s += hist[top - j];
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - s;
+      if (excl < n0 && n0 <= incl) {
+        int acc = excl;
+        for (int j = 1; j <= kPerLane; ++j) {
+          const int c = hist[top - j];
+          if (acc + c >= n0) {
+            scratch[40] = top - j;  // cut bucket
+            scratch[41] = n0 - acc; // members of it to keep
+            break;
+          }
+          acc += c;
+        }
+      }
+      if (lane == 0) scratch[42] = 0;  // member count
+    }
+    __syncthreads();
+    const int cut = scratch[40], want = scratch[41];
+    for (int i = tid; i < ncand; i += kThreads) {
+      if (bkt[i] == cut) mem[atomicAdd(&scratch[42], 1)] = i;
+    }
+    __syncthreads();
+    const int nmem = scratch[42];
+    // exact rank of every member among the members: (score desc, start asc);
+    // candidates are in ascending start order, so start order = index order
+    for (int m = tid; m < nmem; m += kThreads) {
+      const int i = mem[m];
+      const float s = sc[i];
+      int r = 0;
+      for (int x = 0; x < nmem; ++x) {
+        const int jx = mem[x];
+        const float t = sc[jx];
+        r += (t > s || (t == s && jx < i)) ? 1 : 0;
+      }
+      keep[i] = r < want ? 1 : 0;
+    }
+    __syncthreads();
+    // order-preserving compaction of the kept candidates into the chunk list
     const int per_c = (ncand + kThreads - 1) / kThreads;
     const int lo_c = min(ncand, tid * per_c), hi_c = min(ncand, lo_c + per_c);
-    int packed = 0;
-    for (int i = lo_c; i < hi_c; ++i)
-      packed += (keys[i] > theta ? 1 : 0) + (keys[i] == theta ? (1 << 16) : 0);
-    int tot;
-    int run = block_excl_scan(packed, scratch, tot);
+    int nk = 0;
     for (int i = lo_c; i < hi_c; ++i) {
-      const int gt_before = run & 0xffff, eq_before = run >> 16;
-      const bool gt = keys[i] > theta, eq = keys[i] == theta;
-      if (gt || (eq && eq_before < want)) {
-        const int dst = gt_before + min(eq_before, want);
+      const int bi = bkt[i];
+      nk += (bi > cut || (bi == cut && keep[i])) ? 1 : 0;
+    }
+    int total;
+    int dst = block_excl_scan(nk, scratch, total);
+    for (int i = lo_c; i < hi_c; ++i) {
+      const int bi = bkt[i];
+      if (bi > cut || (bi == cut && keep[i])) {
         chunk_s[dst] = cand_s[i];
         chunk_e[dst] = cand_e[i];
+        ++dst;
       }
-      run += (gt ? 1 : 0) + (eq ? (1 << 16) : 0);
+      hist[bi] = 0;  // clear for the next round (each touched bucket)
     }
     __syncthreads();
     buf ^= 1;
@@ -358,45 +430,45 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   // ---- union with sink and window blocks, write the idx row (CTA 0)
   if (rank == 0) {
     const int64_t ns = min64((a.sink + bk - 1) / bk, N);
-    const int64_t cut = a.window > 0 ? max64(0, q_first - a.window + 1) / bk : N;
-    const int64_t lead = min(ns, cut);
-    // kept blocks in [ns, cut): chunk_s is ascending
-    int lo = 0, hi = n0;
+    const int64_t cutb = a.window > 0 ? max64(0, q_first - a.window + 1) / bk : N;
+    const int64_t lead = min64(ns, cutb);
+    int lo_i = 0, hi_i = n0;
     {
       int l = 0, h = n0;
       while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < ns) l = m + 1; else h = m; }
-      lo = l;
-      l = lo; h = n0;
-      while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < cut) l = m + 1; else h = m; }
-      hi = l;
+      lo_i = l;
+      l = lo_i; h = n0;
+      while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < cutb) l = m + 1; else h = m; }
+      hi_i = l;
     }
-    const int64_t mid = hi > lo ? hi - lo : 0;
-    const int64_t tail = a.window > 0 ? N - cut : 0;
+    const int64_t mid = hi_i > lo_i ? hi_i - lo_i : 0;
+    const int64_t tail = a.window > 0 ? N - cutb : 0;
     const int64_t nnz = lead + mid + tail;
     int32_t* row = a.idx + unit * a.row_stride;
     for (int64_t t = tid; t < a.row_stride; t += kThreads) {
       int64_t val;
-      if (t == 0) val = nnz;
-      else {
+      if (t == 0) {
+        val = nnz;
+      } else {
         const int64_t e = t - 1;
         if (e < lead) val = e;
-        else if (e < lead + mid) val = chunk_s[lo + (e - lead)];
-        else if (e < nnz) val = cut + (e - lead - mid);
+        else if (e < lead + mid) val = chunk_s[lo_i + (e - lead)];
+        else if (e < nnz) val = cutb + (e - lead - mid);
         else val = -1;
       }
       row[t] = static_cast<int32_t>(val);
     }
   }
-  if (timed_out) report(status, kStatusTimeout, 1);
-  cluster.sync();  // peers may still read this CTA's scores
+  if (timed_out) report(a.status, kStatusTimeout, 1);
+  if (C > 1) cluster.sync();  // peers may still read this CTA's scores
 }
 
 template <typename T, int RC>
-cudaError_t launch_mask_t(const MaskArgs& a, int smem, cudaStream_t stream) {
-  auto kern = mask_fma_kernel<T, RC>;
-  // attributes are set once per kernel (not inside a later stream capture)
+cudaError_t prepare_t(const MaskArgs& a, int smem) {
+  // attributes are set once per kernel and device (not inside a stream capture)
   static int smem_set[kMaxDevices] = {};
   static bool big_cluster_set[kMaxDevices] = {};
+  auto kern = mask_fma_kernel<T, RC>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -411,19 +483,49 @@ cudaError_t launch_mask_t(const MaskArgs& a, int smem, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     big_cluster_set[dev] = true;
   }
+  return cudaSuccess;
+}
+
+template <typename T, int RC>
+cudaLaunchConfig_t config_t(const MaskArgs& a, int smem, cudaStream_t stream,
+                            cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.cluster, static_cast<unsigned>(a.units), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = a.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return cfg;
+}
+
+template <typename T, int RC>
+cudaError_t launch_mask_t(const MaskArgs& a, int smem, cudaStream_t stream) {
+  cudaError_t e = prepare_t<T, RC>(a, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = config_t<T, RC>(a, smem, stream, attr);
+  return cudaLaunchKernelEx(&cfg, mask_fma_kernel<T, RC>, a);
+}
+
+template <typename T, int RC>
+int max_active_clusters_t(const MaskArgs& a, int smem) {
+  if (prepare_t<T, RC>(a, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = config_t<T, RC>(a, smem, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, mask_fma_kernel<T, RC>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  return n;
 }
 
 template <typename T>
@@ -435,15 +537,28 @@ cudaError_t launch_mask_rc(const MaskArgs& a, int smem, cudaStream_t s) {
   return launch_mask_t<T, 8>(a, smem, s);
 }
 
+template <typename T>
+int max_active_rc(const MaskArgs& a, int smem) {
+  const int R = a.rows_max;
+  if (R <= 1) return max_active_clusters_t<T, 1>(a, smem);
+  if (R <= 2) return max_active_clusters_t<T, 2>(a, smem);
+  if (R <= 4) return max_active_clusters_t<T, 4>(a, smem);
+  return max_active_clusters_t<T, 8>(a, smem);
+}
+
 }  // namespace
 
 int mask_fma_rc(int rows_max) { return rows_max <= 1 ? 1 : rows_max <= 2 ? 2 : rows_max <= 4 ? 4 : 8; }
 
-int mask_fma_smem_bytes(int n0max, int rows_pad, int per_cta) {
-  return mask_smem_layout(n0max, rows_pad, per_cta).total;
+int mask_fma_smem_bytes(int n0max, int rows_pad, int per_cta, int cluster, int stages) {
+  return mask_smem_layout(n0max, rows_pad, per_cta, cluster, stages).total;
 }
 
 int mask_fma_tile_keys(int dtype) { return kTileBytes / (dtype == 1 ? 256 : 512); }
+
+int mask_fma_max_active_clusters(const MaskArgs& a, int smem) {
+  return a.dtype == 1 ? max_active_rc<uint16_t>(a, smem) : max_active_rc<float>(a, smem);
+}
 
 cudaError_t launch_mask_fma(const MaskArgs& a, int smem, cudaStream_t stream) {
   return a.dtype == 1 ? launch_mask_rc<uint16_t>(a, smem, stream)

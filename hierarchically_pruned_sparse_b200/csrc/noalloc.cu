@@ -15,7 +15,8 @@
 namespace {
 
 constexpr size_t kScratchBytes = HIPS_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kStatusBytes = 256;
+constexpr size_t kStatusBytes = 4096;  // status word + split-merge counters
+constexpr size_t kCounterOffset = 256;
 
 // One copy per device that loads the library, alive until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -56,10 +57,12 @@ extern "C" int hip_sparse_attn_noalloc(const void* q, const void* k, const void*
   st = scratch_on_current_device(&base);
   if (st) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
-  // the status block must start at zero; the partials are fully overwritten
+  // the status word and the split-merge counters must start at zero; the
+  // partials are fully overwritten
   cudaError_t e = cudaMemsetAsync(base, 0, kStatusBytes, stream);
   if (e != cudaSuccess) return hips::record_cuda_error(e);
   a.status = static_cast<hips::Status*>(base);
+  a.counters = reinterpret_cast<unsigned int*>(static_cast<unsigned char*>(base) + kCounterOffset);
   a.part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kStatusBytes);
   return hips::record_cuda_error(hips::launch_attn_fma(a, smem, stream));
 }

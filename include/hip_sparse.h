@@ -42,9 +42,12 @@
  *    at absolute position q_pos0 + i and sees keys j <= q_pos0 + i.
  *  - head_dim must be 128. k, v, q, out must be 16-byte aligned.
  *  - Every call needs a workspace of at least hip_workspace_size(params, op)
- *    bytes (256-byte aligned, caller-owned). Its first 256 bytes are a sticky
- *    status block: kernels only ever set bits there. Clear it once after
- *    allocating (hip_workspace_init) and read it with hip_check_status.
+ *    bytes (256-byte aligned, caller-owned). Its first 4096 bytes are a
+ *    status block: a sticky error word (kernels only ever set bits there) and
+ *    the split-merge counters of the attention, which are zero between
+ *    calls. Clear it once after allocating (hip_workspace_init) and read it
+ *    with hip_check_status. Calls sharing one workspace must not overlap on
+ *    the GPU (issue them on one stream).
  *  - Return value: HIPS_OK (0) or a negative HIPS_ERR_* code. Argument errors
  *    are found on the host before anything is launched. HIPS_ERR_CUDA means
  *    a launch failed; hip_last_cuda_error() gives the cudaError_t.
@@ -109,7 +112,7 @@ HIPS_API int64_t hip_idx_row_stride(const hips_params* params);
  * params; 0 if the params are invalid. */
 HIPS_API size_t hip_workspace_size(const hips_params* params, int op);
 
-/* Zero the status block of params->workspace (async on params->stream). */
+/* Zero the 4096-byte status block of params->workspace (async on params->stream). */
 HIPS_API int hip_workspace_init(const hips_params* params);
 
 /* Synchronise params->stream, read and clear the status block. Returns
@@ -152,7 +155,7 @@ HIPS_API int hip_dense_attn(const void* q, const void* k, const void* v, const h
  *    it: serialise them.
  *  - Bounded-wait failures of this call are not reported through
  *    hip_check_status (it has no caller workspace). */
-#define HIPS_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define HIPS_NOALLOC_SCRATCH_BYTES (512u << 10)
 HIPS_API int hip_sparse_attn_noalloc(const void* q, const void* k, const void* v,
                                      const int32_t* idx, const hips_params* params, void* out);
 

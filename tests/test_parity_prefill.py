@@ -1,0 +1,93 @@
+"""GPU parity of the prefill mask (query blocks of b_q rows scored on tensor
+cores with the exact re-score band) against the oracle."""
+import functools
+
+import numpy as np
+import pytest
+
+import oracle
+from hierarchically_pruned_sparse_b200 import workloads as W
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    import torch
+    from hierarchically_pruned_sparse_b200 import build
+    assert torch.cuda.is_available(), "gpu tests need a CUDA device"
+    build.build()
+    oracle.set_threads(0)
+
+
+@functools.lru_cache(maxsize=2)
+def _inputs(w: W.Workload):
+    return W.make_inputs(w)
+
+
+def _gpu_mask(w, x):
+    import torch
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    osh, bkw = pu.shapes(w)
+    q, k, _ = pu.torch_inputs(x, w)
+    s = hb.Session(**bkw)
+    idx = s.mask(q, k)
+    torch.cuda.synchronize()
+    s.check()
+    return osh, idx.cpu().numpy().reshape(-1, idx.shape[-1])
+
+
+SMALL = [
+    # 4 heads x 64 positions = 256 rows per mask, ragged last query block
+    W.Workload("p256", "prefill", 1, 4, 1, 128, 3000, 64, 2, 256, 16, 64, "bf16"),
+    # 2 heads x 64 = 128 rows, 4-key blocks, two KV heads, batch 2
+    W.Workload("p128", "prefill", 2, 4, 2, 128, 2100, 64, 4, 256, 0, 0, "bf16"),
+    # 1 head x 64 = 64 rows, one-key blocks
+    W.Workload("p64", "prefill", 1, 1, 1, 128, 1500, 64, 1, 128, 4, 32, "bf16"),
+    # 16-key blocks, 8 rows per mask (b_q = 2, 4 heads)
+    W.Workload("p8", "prefill", 1, 4, 1, 128, 1200, 2, 16, 256, 0, 16, "bf16"),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_prefill_mask(w):
+    x = _inputs(w)
+    osh, got = _gpu_mask(w, x)
+    ref, gap, _ = oracle.mask(x["q"][0], x["k"], osh)
+    pu.compare_masks(got, ref, gap)
+
+
+def test_prefill_32k_mask_sampled():
+    w = W.PREFILL_32K
+    x = _inputs(w)
+    osh, got = _gpu_mask(w, x)
+    nqb = oracle.num_qblocks(osh)
+    rng = np.random.default_rng(0)
+    qbs = sorted(set([0, 31, 32, 33, 200, nqb - 1]) | set(rng.choice(nqb, 10, replace=False).tolist()))
+    units = np.array([g * nqb + qb for g in range(w.n_kvheads) for qb in qbs if (g + qb) % 3 == 0]
+                     + [g * nqb + nqb - 1 for g in range(w.n_kvheads)], dtype=np.int64)
+    units = np.unique(units)
+    ref, gap, _ = oracle.mask(x["q"][0], x["k"], osh, units=units)
+    pu.compare_masks(got[units], ref, gap)
+
+
+def test_equal_keys_every_candidate_in_the_band():
+    # every score ties: the whole candidate set is re-scored canonically and
+    # the tie rule keeps the lowest blocks
+    import torch
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    T, bk, topk = 4096, 2, 256
+    rng = np.random.default_rng(0)
+    q = W.bf16_round(rng.standard_normal((1, 4, 1, 128)).astype(np.float32))
+    k = np.ascontiguousarray(np.broadcast_to(W.bf16_round(rng.standard_normal(128).astype(np.float32)),
+                                             (1, 1, T, 128)))
+    s = hb.Session(batch=1, n_qheads=4, n_kvheads=1, seq_len=T, q_len=1, q_pos0=T - 1,
+                   dtype=hb.HIPS_BF16, block_q=1, block_k=bk, topk=topk)
+    idx = s.mask(torch.from_numpy(q).cuda().to(torch.bfloat16).contiguous(),
+                 torch.from_numpy(k).cuda().to(torch.bfloat16).contiguous())
+    torch.cuda.synchronize()
+    s.check()
+    got = idx.cpu().numpy().reshape(-1)
+    assert got[0] == topk // bk
+    assert list(got[1:1 + got[0]]) == list(range(topk // bk))

@@ -57,7 +57,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_refuses_requests_beyond_its_array():
     # 64 query heads over 8 KV heads at 128k: the split-K partials of 64 rows
-    # (about 1.2 MB) need more than the 1 MiB array holds
+    # (about 0.6 MB) need more than the 512 KiB array holds
     big = hb.params(batch=1, n_qheads=64, n_kvheads=8, seq_len=131072, q_len=1,
                     q_pos0=131071, dtype=hb.HIPS_BF16, block_q=1, block_k=2, topk=2048,
                     sink=128, window=1024)
