@@ -77,8 +77,15 @@ int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
     return HIPS_ERR_UNSUPPORTED;
   const int cpt = hips::mask_mma_tile_keys() / p->block_k;
   const int64_t ncand = 2 * static_cast<int64_t>(a.n0max);
+  // the largest cluster (any size up to the cap) with one CTA per SM for all
+  // units and at least one full tile of candidates per CTA
   int c = 1;
-  while (c < cluster_cap && a.units * (2 * c) <= kPlanSMs && cdiv(ncand, 2 * c) >= cpt) c *= 2;
+  for (int t = std::min(cluster_cap, 16); t > 1; --t) {
+    if (a.units * t <= kPlanSMs && cdiv(ncand, t) >= cpt) {
+      c = t;
+      break;
+    }
+  }
   a.cluster = c;
   a.per_cta = static_cast<int>(cdiv(ncand, c));
   a.rows_pad = nc * 16;
@@ -120,7 +127,7 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   const int cpt = tile_keys / p->block_k;
   const int64_t ncand = 2 * static_cast<int64_t>(a.n0max);
   int c = 1;
-  while (c < cluster_cap && a.units * (2 * c) <= kPlanSMs && cdiv(ncand, 2 * c) >= cpt) c *= 2;
+  while (2 * c <= cluster_cap && a.units * (2 * c) <= kPlanSMs && cdiv(ncand, 2 * c) >= cpt) c *= 2;
   a.cluster = c;
   a.per_cta = static_cast<int>(cdiv(ncand, c));
   a.stages = 3;
@@ -162,12 +169,40 @@ struct AttnPlan {
   hips::AttnArgs a;
   int smem;
   size_t ws;
+  bool mma;  // tensor-core kernel (query blocks, bf16) or CUDA-core split-K kernel
 };
+
+// Tensor-core plan: bf16 query blocks of more than 8 rows (a CTA per 128 rows
+// of a block, every key of the row list in one CTA).
+int plan_attn_mma(const hips_params* p, bool dense, AttnPlan* plan) {
+  hips::AttnArgs& a = plan->a;
+  if (p->dtype != HIPS_BF16 || a.rows_max <= 8) return HIPS_ERR_UNSUPPORTED;
+  a.item_keys = dense ? 16 : p->block_k;
+  if (a.item_keys > hips::attn_mma_tile_keys()) return HIPS_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(a.nqb) * p->n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
+  int64_t items;
+  if (dense) {
+    items = cdiv(std::min<int64_t>(p->q_pos0 + p->q_len, p->seq_len), a.item_keys);
+  } else {
+    items = (a.row_stride - 1) + cdiv(std::max<int64_t>(0, p->seq_len - p->mask_len), a.item_keys);
+  }
+  if (items > (1 << 20)) return HIPS_ERR_UNSUPPORTED;
+  a.table_items = static_cast<int>(items);
+  a.nsplit = 1;
+  plan->smem = hips::attn_mma_smem_bytes(a.table_items);
+  if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
+  plan->mma = true;
+  plan->ws = kStatusBytes;
+  return HIPS_OK;
+}
 
 int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
   hips::AttnArgs& a = plan->a;
   a = hips::AttnArgs{};
-  const int block_q = dense ? 1 : p->block_q;
+  plan->mma = false;
+  // dense prefill (bf16) runs on the tensor-core kernel in 64-row query blocks
+  const bool dense_blocks = dense && p->dtype == HIPS_BF16 && p->q_len >= 64;
+  const int block_q = dense ? (dense_blocks ? 64 : 1) : p->block_q;
   a.dtype = p->dtype;
   a.batch = p->batch;
   a.n_qheads = p->n_qheads;
@@ -185,6 +220,7 @@ int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
   a.row_stride = dense ? 0 : row_stride(p);
   a.rows_total = static_cast<int64_t>(p->batch) * p->n_qheads * p->q_len;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
+  if (plan_attn_mma(p, dense, plan) == HIPS_OK) return HIPS_OK;
   if (a.rows_max > 8) return HIPS_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(a.nqb) * p->n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
   a.item_keys = dense ? 16 : p->block_k;
@@ -242,7 +278,9 @@ int run_attention(const void* q, const void* k, const void* v, const int32_t* id
   a.status = static_cast<hips::Status*>(p->workspace);
   a.part = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + kStatusBytes);
   a.counters = reinterpret_cast<unsigned int*>(static_cast<char*>(p->workspace) + kCounterOffset);
-  return cuda_status(hips::launch_attn_fma(a, plan.smem, static_cast<cudaStream_t>(p->stream)));
+  cudaStream_t stream = static_cast<cudaStream_t>(p->stream);
+  return cuda_status(plan.mma ? hips::launch_attn_mma(a, plan.smem, stream)
+                              : hips::launch_attn_fma(a, plan.smem, stream));
 }
 
 }  // namespace
@@ -253,7 +291,7 @@ namespace hips {
 // scratch memory (no caller workspace); *scratch_bytes is what it needs.
 int plan_sparse_attn_own_scratch(const void* q, const void* k, const void* v, const int32_t* idx,
                                  const hips_params* p, void* out, AttnArgs* args, int* smem,
-                                 size_t* scratch_bytes) {
+                                 size_t* scratch_bytes, bool* tensor_core) {
   int st = validate(p, HIPS_OP_SPARSE);
   if (st) return st;
   if (!q || !k || !v || !out || !idx) return HIPS_ERR_INVALID_ARG;
@@ -267,6 +305,7 @@ int plan_sparse_attn_own_scratch(const void* q, const void* k, const void* v, co
   args->q = q; args->k = k; args->v = v; args->idx = idx; args->out = out;
   *smem = plan.smem;
   *scratch_bytes = plan.ws;
+  *tensor_core = plan.mma;
   return HIPS_OK;
 }
 
@@ -328,7 +367,7 @@ int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* i
   // A cluster of C CTAs needs C free SMs of one GPC. Take the largest cluster
   // for which every mask row is resident at once (one wave); fall back to
   // smaller clusters if the device refuses the shape.
-  for (int cap = 16; cap >= 1; cap /= 2) {
+  for (int cap = 16; cap >= 1; cap = std::min(cap - 1, plan.a.cluster - 1)) {
     st = plan_mask(params, cap, &plan);
     if (st) return st;
     if (plan.a.cluster > cap) continue;

@@ -9,10 +9,10 @@
 // key in [mask_len, seq_len) appended since the mask was computed (the mask
 // refresh interval r_m of the research-map summary, Limitations).
 //
-// Design: grid (splits, KV head x query block, sequence). A split takes a
-// contiguous range of work items (one key block each); K and V rows of a
+// Design: grid (splits, KV head x query block, sequence). Split s takes the
+// work items s, s + splits, ... (one key block each); K and V rows of a
 // 64-key tile are gathered by all threads with 16-byte cp.async copies into a
-// 3-stage ring (completion tracked on one mbarrier per stage), the
+// 3-stage ring (all stages requested up front) (completion tracked on one mbarrier per stage), the
 // G query heads of the group share every gathered tile, and each of 8 warps
 // works on 4 keys at a time with 8 lanes per key (16 head elements per lane).
 // Scores go through an fp32 online softmax (exp2 domain); each split writes
@@ -106,30 +106,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   // the idx rows may come from the kernel launched just before this one
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- work items of this unit and this split's range
+  // ---- work items of this split: items split, split + nsplit, ... (strided,
+  // so the splits stay balanced whatever nnz is). nnz and this split's block
+  // ids are loaded together (one memory latency); ids are range-checked so a
+  // malformed row cannot drive reads outside [0, seq_len)
   const int64_t unit = (static_cast<int64_t>(b) * a.n_kvheads + g) * a.nqb + qb;
   const int32_t* idx_row = a.dense ? nullptr : a.idx + unit * a.row_stride;
-  int64_t nitems;
-  int nnz = 0;
-  if (a.dense) {
-    const int64_t Tc = min(q_last + 1, a.seq_len);
-    nitems = (Tc + IK - 1) / IK;
-  } else {
-    nnz = max(0, min(idx_row[0], static_cast<int>(a.row_stride - 1)));
-    const int64_t tail = max64(0, a.seq_len - a.mask_len);
-    nitems = nnz + (tail + IK - 1) / IK;
-  }
-  const int64_t per = (nitems + a.nsplit - 1) / a.nsplit;
-  const int64_t it_lo = min(nitems, split * per), it_hi = min(nitems, it_lo + per);
-  const int nmine = static_cast<int>(it_hi - it_lo);
-
-  // item table (sparse): first key and key count of every item of this split;
-  // ids read from idx are range-checked so a malformed row cannot drive reads
-  // outside [0, seq_len)
   const int64_t vis = min64(q_last + 1, a.seq_len);
-  if (!a.dense) {
-    for (int t = tid; t < nmine; t += kThreads) {
-      const int64_t it = it_lo + t;
+  int nmine;
+  if (a.dense) {
+    const int64_t nitems = (vis + IK - 1) / IK;
+    nmine = nitems > split ? static_cast<int>((nitems - split + a.nsplit - 1) / a.nsplit) : 0;
+  } else {
+    const int cap = static_cast<int>(a.row_stride - 1);
+    const int64_t tail_items = (max64(0, a.seq_len - a.mask_len) + IK - 1) / IK;
+    const int raw_nnz = idx_row[0];
+    int raw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t it = split + static_cast<int64_t>(a.nsplit) * (tid + u * kThreads);
+      raw[u] = (tid + u * kThreads < a.table_items && it < cap) ? idx_row[1 + it] : -1;
+    }
+    const int nnz = max(0, min(raw_nnz, cap));
+    const int64_t nitems = nnz + tail_items;
+    nmine = nitems > split ? static_cast<int>((nitems - split + a.nsplit - 1) / a.nsplit) : 0;
+    nmine = min(nmine, a.table_items);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int t = tid + u * kThreads;
+      if (t < nmine) {
+        const int64_t it = split + static_cast<int64_t>(a.nsplit) * t;
+        int64_t j0, n;
+        if (it < nnz) {
+          const int64_t c = raw[u];
+          j0 = c * IK;
+          n = c < 0 ? 0 : min64(IK, min64(a.mask_len, vis) - j0);
+        } else {
+          j0 = a.mask_len + (it - nnz) * IK;
+          n = min64(IK, vis - j0);
+        }
+        table[t] = make_int2(static_cast<int>(max64(j0, 0)), static_cast<int>(max64(n, 0)));
+      }
+    }
+    for (int t = tid + 2 * kThreads; t < nmine; t += kThreads) {  // long rows (few splits)
+      const int64_t it = split + static_cast<int64_t>(a.nsplit) * t;
       int64_t j0, n;
       if (it < nnz) {
         const int64_t c = idx_row[1 + it];
@@ -144,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   }
   auto item_at = [&](int t) -> int2 {
     if (!a.dense) return table[t];
-    const int64_t j0 = (it_lo + t) * IK;
+    const int64_t j0 = (split + static_cast<int64_t>(a.nsplit) * t) * IK;
     return make_int2(static_cast<int>(j0), static_cast<int>(max64(min64(IK, vis - j0), 0)));
   };
   __syncthreads();
@@ -183,10 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   float m_run = -INFINITY, l_run = 0.0f;  // valid in warp r for row r
   bool timed_out = false;
 
-  for (int t = 0; t < min(kStages - 1, ntiles); ++t) issue(t);
+  for (int t = 0; t < min(kStages, ntiles); ++t) issue(t);
 
   for (int t = 0; t < ntiles; ++t) {
-    if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
     const int slot = t % kStages;
     if (!mbar_wait(&bars[slot], (t / kStages) & 1)) timed_out = true;
     const int f = t * ipt, cnt = min(ipt, nmine - f);
@@ -270,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
         for (int e = 0; e < 16; ++e) acc[r][e] = __fmaf_rn(pk[r], vx[e], acc[r][e]);
     }
     __syncthreads();
+    if (t + kStages < ntiles) issue(t + kStages);  // into the slot just consumed
   }
 
   // ---- reduce the 4 key groups of a warp, then the 8 warps

@@ -50,6 +50,12 @@ int mask_mma_tile_keys();
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream);
 
+// Tensor-core attention for query blocks, bf16 (attn_mma.cu)
+int attn_mma_smem_bytes(int table_items);
+int attn_mma_tile_keys();
+int attn_mma_rows();
+cudaError_t launch_attn_mma(const AttnArgs& a, int smem, cudaStream_t stream);
+
 // CUDA-core split-K attention with the split merge fused (attn_fma.cu)
 int attn_fma_tile_keys(int dtype);
 int attn_fma_smem_bytes(int dtype, int rows_max, int table_items);
@@ -59,7 +65,7 @@ cudaError_t launch_attn_fma(const AttnArgs& a, int smem, cudaStream_t stream);
 // (api.cu); the no-allocation entry point in noalloc.cu launches it.
 int plan_sparse_attn_own_scratch(const void* q, const void* k, const void* v, const int32_t* idx,
                                  const hips_params* p, void* out, AttnArgs* args, int* smem,
-                                 size_t* scratch_bytes);
+                                 size_t* scratch_bytes, bool* tensor_core);
 int record_cuda_error(cudaError_t e);
 
 }  // namespace hips

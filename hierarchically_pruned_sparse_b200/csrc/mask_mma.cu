@@ -45,19 +45,21 @@ constexpr int kM = 128;                 // keys per MMA tile
 constexpr int kTileBytes = kM * 256;    // bf16 key rows
 constexpr int kHalfBytes = kTileBytes / 2;
 constexpr int kBuckets = 2048;
-constexpr int kMaxPer = (2 * kMaxN0 + kThreads - 1) / kThreads;
 constexpr float kGamma = 1024.0f / 16777216.0f;
 
-__host__ __device__ constexpr int stages_for(int nc) { return nc >= 16 ? 2 : 3; }
+__host__ __device__ constexpr int stages_for(int nc) { return nc >= 16 ? 2 : nc >= 8 ? 3 : 4; }
 __host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 16 < 32 ? 32 : nc * 16; }
 
 struct MmaSmem {
-  int ring, bq, bar, slot, chunk_s, chunk_e, cand_s, cand_e, sc_t, sc_e, bkt, cls, mem, band,
-      band_key, xch, hist, scratch, total;
+  int ring, bq, bar, slot, cs, ce, keepb, band, band_key, xch, hist, scratch, total;
 };
 
 __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
 
+// cs/ce (candidate start and end block) are double-buffered: a round reads one
+// copy and writes the next round's list into the other. xch holds the (score,
+// bound) of every candidate of a round: each CTA writes its own candidates
+// into every CTA of the cluster; two copies alternate between rounds.
 __host__ __device__ inline MmaSmem mma_layout(int nc, int n0max, int per_cta, int cluster) {
   MmaSmem L;
   const int n = 2 * n0max;
@@ -66,27 +68,27 @@ __host__ __device__ inline MmaSmem mma_layout(int nc, int n0max, int per_cta, in
   L.bq = o;       o += nc * 16 * 256;
   L.bar = o;      o += 16;
   L.slot = o;     o += 16;
-  L.chunk_s = o;  o += al(n0max * 4, 16);
-  L.chunk_e = o;  o += al(n0max * 4, 16);
-  L.cand_s = o;   o += al(n * 4, 16);
-  L.cand_e = o;   o += al(n * 4, 16);
-  L.sc_t = o;     o += al(n * 4, 16);
-  L.sc_e = o;     o += al(n * 4, 16);
-  L.bkt = o;      o += al(n * 2, 16);
-  L.cls = o;      o += al(n, 16);
-  L.mem = o;      o += al(n * 4, 16);
+  L.cs = o;       o += 2 * al(n * 4, 16);
+  L.ce = o;       o += 2 * al(n * 4, 16);
+  L.keepb = o;    o += al(n, 16);
   L.band = o;     o += al(n * 4, 16);
   L.band_key = o; o += al(n * 4, 16);
-  L.xch = o;      o += cluster > 1 ? al(2 * per_cta * 8, 16) : 0;
+  L.xch = o;      o += (cluster > 1 ? 2 : 1) * al(n * 8, 16);
+  (void)per_cta;
   L.hist = o;     o += kBuckets * 4;
   L.scratch = o;  o += 64 * 4;
   L.total = o + 1024;  // room to align the base to 1024 bytes
   return L;
 }
 
+__device__ __forceinline__ float key_score(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(u);
+}
+
 // Cut bucket of the n-th largest (1-based) under a histogram of kBuckets bins:
 // every thread owns 8 consecutive bins, thread 0 the top ones.
-__device__ void find_cut(const int* hist, int n, int* scratch, int* cut, int* want) {
+__device__ int find_cut(const int* hist, int n, int* scratch) {
   const int top = kBuckets - 8 * threadIdx.x;
   int c[8], s = 0;
 #pragma unroll
@@ -100,19 +102,15 @@ __device__ void find_cut(const int* hist, int n, int* scratch, int* cut, int* wa
     int acc = before;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (acc < n && n <= acc + c[j]) {
-        scratch[40] = top - 1 - j;
-        scratch[41] = n - acc;
-      }
+      if (acc < n && n <= acc + c[j]) scratch[40] = top - 1 - j;
       acc += c[j];
     }
   }
   __syncthreads();
-  *cut = scratch[40];
-  *want = scratch[41];
+  return scratch[40];
 }
 
-template <int NC>
+template <int NC, int PER>
 __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   constexpr int N = NC * 16;
   constexpr int S = stages_for(NC);
@@ -138,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   const int64_t N_blocks = (Tc + bk - 1) / bk;
   const int n0 = static_cast<int>(min64(a.n0max, N_blocks));
   const int per_cta = a.per_cta;
+  const int nbuf = 2 * a.n0max;  // stride between the two candidate buffers
 
   const MmaSmem L = mma_layout(NC, a.n0max, per_cta, C);
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -145,21 +144,16 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   unsigned char* bq = smem + L.bq;
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.slot);
-  int* chunk_s = reinterpret_cast<int*>(smem + L.chunk_s);
-  int* chunk_e = reinterpret_cast<int*>(smem + L.chunk_e);
-  int* cand_s = reinterpret_cast<int*>(smem + L.cand_s);
-  int* cand_e = reinterpret_cast<int*>(smem + L.cand_e);
-  float* sc_t = reinterpret_cast<float*>(smem + L.sc_t);
-  float* sc_e = reinterpret_cast<float*>(smem + L.sc_e);
-  uint16_t* bkt = reinterpret_cast<uint16_t*>(smem + L.bkt);
-  uint8_t* cls = reinterpret_cast<uint8_t*>(smem + L.cls);
-  int* mem = reinterpret_cast<int*>(smem + L.mem);
+  int* cs_all = reinterpret_cast<int*>(smem + L.cs);
+  int* ce_all = reinterpret_cast<int*>(smem + L.ce);
+  uint8_t* keepb = reinterpret_cast<uint8_t*>(smem + L.keepb);
   int* band = reinterpret_cast<int*>(smem + L.band);
   uint32_t* band_key = reinterpret_cast<uint32_t*>(smem + L.band_key);
   float2* xch = reinterpret_cast<float2*>(smem + L.xch);
   int* hist = reinterpret_cast<int*>(smem + L.hist);
   int* scratch = reinterpret_cast<int*>(smem + L.scratch);
   float* fscratch = reinterpret_cast<float*>(scratch);
+  uint32_t* uscratch = reinterpret_cast<uint32_t*>(scratch);
 
   const uint16_t* qg = static_cast<const uint16_t*>(a.q);
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
@@ -183,6 +177,41 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     }
     *reinterpret_cast<uint4*>(bq + (c >> 3) * (N * 128) + sw128_offset(r, c & 7)) = v;
   }
+  for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
+
+  // ---- candidates of round 1: the halves of the n0 initial chunks
+  // (a one-block chunk stays whole); thread t owns chunks [t*pc, (t+1)*pc)
+  int ncand, nlong;
+  {
+    const int pc = (n0 + kThreads - 1) / kThreads;
+    const int lo = min(n0, tid * pc), hi = min(n0, lo + pc);
+    int cnt = 0, nl = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int64_t s0 = static_cast<int64_t>(i) * N_blocks / n0;
+      const int64_t e0 = static_cast<int64_t>(i + 1) * N_blocks / n0;
+      cnt += e0 - s0 > 1 ? 2 : 1;
+      nl += e0 - s0 > 1 ? 1 : 0;
+    }
+    int tot;
+    int pos = block_excl_scan(cnt | (nl << 16), scratch, tot) & 0xffff;
+    ncand = tot & 0xffff;
+    nlong = tot >> 16;
+    for (int i = lo; i < hi; ++i) {
+      const int s0 = static_cast<int>(static_cast<int64_t>(i) * N_blocks / n0);
+      const int e0 = static_cast<int>(static_cast<int64_t>(i + 1) * N_blocks / n0);
+      auto put = [&](int s, int e) {
+        cs_all[pos] = s;
+        ce_all[pos] = e;
+        ++pos;
+      };
+      if (e0 - s0 > 1) {
+        put(s0, s0 + (e0 - s0) / 2);
+        put(s0 + (e0 - s0) / 2, e0);
+      } else {
+        put(s0, e0);
+      }
+    }
+  }
   // max over the rows of sum_i |q_ri| (rounded up)
   float q1 = 0.0f;
   for (int r = tid; r < R; r += kThreads) {
@@ -195,11 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) q1 = fmaxf(q1, __shfl_xor_sync(0xffffffffu, q1, o));
   if (lane == 0) fscratch[48 + warp] = q1;
-  for (int i = tid; i < n0; i += kThreads) {
-    chunk_s[i] = static_cast<int>(static_cast<int64_t>(i) * N_blocks / n0);
-    chunk_e[i] = static_cast<int>(static_cast<int64_t>(i + 1) * N_blocks / n0);
-  }
-  for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
   fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
@@ -210,66 +234,48 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   for (int w = 1; w < kWarps; ++w) q1max = fmaxf(q1max, fscratch[48 + w]);
   const float eps_scale = kGamma * q1max;
   const uint32_t idesc = idesc_bf16_f32(kM, N);
-  const int cpt = kM / bk;  // candidates per tile
+  const int cpt = kM >> lbk;  // candidates per tile
   uint32_t mma_phase = 0;
-  int buf = 0;
+  int cur = 0, buf = 0;
   bool timed_out = false;
 
-  for (;;) {
-    // ---- candidates: halves of every chunk; a one-block chunk stays whole
-    const int per_t = (n0 + kThreads - 1) / kThreads;
-    const int lo_t = min(n0, tid * per_t), hi_t = min(n0, lo_t + per_t);
-    int cnt = 0, nlong = 0;
-    for (int i = lo_t; i < hi_t; ++i) {
-      const int len = chunk_e[i] - chunk_s[i];
-      cnt += len > 1 ? 2 : 1;
-      nlong += len > 1 ? 1 : 0;
-    }
-    int tot;
-    int pos = block_excl_scan(cnt | (nlong << 16), scratch, tot);
-    if ((tot >> 16) == 0) break;
-    const int ncand = tot & 0xffff;
-    pos &= 0xffff;
-    for (int i = lo_t; i < hi_t; ++i) {
-      const int s = chunk_s[i], e = chunk_e[i], len = e - s;
-      if (len > 1) {
-        const int m = s + len / 2;
-        cand_s[pos] = s; cand_e[pos] = m; ++pos;
-        cand_s[pos] = m; cand_e[pos] = e; ++pos;
-      } else {
-        cand_s[pos] = s; cand_e[pos] = e; ++pos;
-      }
-    }
-    __syncthreads();
+  while (nlong > 0) {
+    const int* cs = cs_all + cur * nbuf;
+    const int* ce = ce_all + cur * nbuf;
+    // first key of candidate c's representative (centre) block
+    auto rep_key = [&](int c) -> int64_t {
+      return static_cast<int64_t>(cs[c] + (ce[c] - cs[c]) / 2) << lbk;
+    };
 
     // ---- tensor-core scores of this CTA's candidates
     const int c_lo = min(ncand, rank * per_cta), c_hi = min(ncand, c_lo + per_cta);
     const int ntiles = (c_hi - c_lo + cpt - 1) / cpt;
-    float* my_t = C > 1 ? nullptr : sc_t;
-    float* my_e = C > 1 ? nullptr : sc_e;
-    float2* my_x = C > 1 ? xch + buf * per_cta : nullptr;
+    float2* my_x = xch + buf * nbuf;  // indexed by candidate
 
-    auto issue = [&](int t) {  // all threads: gather tile t (if any) and commit a group
+    // all threads: gather tile t (if any) into its ring slot, commit a group;
+    // thread t copies chunk (t % 16) of keys t/16, t/16 + 16, ... of the tile
+    auto issue = [&](int t) {
       if (t < ntiles) {
         unsigned char* dst = ring + (t % S) * kTileBytes;
-        const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
-        const int nchunks = (cc << lbk) * 16;
-        for (int i = tid; i < nchunks; i += kThreads) {
-          const int kk = i >> 4, ch = i & 15;
-          const int c = cf + (kk >> lbk);
-          const int64_t rep = cand_s[c] + (cand_e[c] - cand_s[c]) / 2;
-          const int64_t j = rep * bk + (kk & (bk - 1));
-          if (j < Tc)
-            cp_async16(dst + (ch >> 3) * kHalfBytes + sw128_offset(kk, ch & 7),
-                       kbase + j * 256 + ch * 16);
+        const int cf = c_lo + t * cpt;
+        const int nkeys = min(cpt, c_hi - cf) << lbk;
+        const int ch = tid & 15;
+        unsigned char* dch = dst + (ch >> 3) * kHalfBytes;
+#pragma unroll
+        for (int m = 0; m < kM / 16; ++m) {
+          const int kk = (tid >> 4) + 16 * m;
+          if (kk < nkeys) {
+            const int64_t j = rep_key(cf + (kk >> lbk)) + (kk & (bk - 1));
+            if (j < Tc) cp_async16(dch + sw128_offset(kk, ch & 7), kbase + j * 256 + ch * 16);
+          }
         }
       }
       cp_async_commit();
     };
 
-    for (int t = 0; t < S - 1; ++t) issue(t);
+    for (int t = 0; t < S; ++t) issue(t);
     for (int t = 0; t < ntiles; ++t) {
-      cp_async_wait<S - 2>();
+      cp_async_wait<S - 1>();
       fence_proxy_async_smem();
       tc_fence_before_sync();
       __syncthreads();
@@ -291,8 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         bool kvalid = lc < cc;
         int64_t j = 0;
         if (kvalid) {
-          const int c = cf + lc;
-          j = (cand_s[c] + (cand_e[c] - cand_s[c]) / 2) * static_cast<int64_t>(bk) + (kk & (bk - 1));
+          j = rep_key(cf + lc) + (kk & (bk - 1));
           kvalid = j < Tc;
         }
         // max |k| of this key row (bf16 magnitudes compare as integers)
@@ -331,46 +336,37 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
           eps = fmaxf(eps, __shfl_xor_sync(0xffffffffu, eps, o));
         }
         if ((kk & (bk - 1)) == 0 && lc < cc) {
-          const int o = cf - c_lo + lc;
-          if (C > 1) my_x[o] = make_float2(tsc, eps);
-          else { my_t[o] = tsc; my_e[o] = eps; }
+          const float2 val = make_float2(tsc, eps);
+          my_x[cf + lc] = val;
+          for (int p = 0; p < C; ++p)  // push to the peers (read after the cluster barrier)
+            if (p != rank) *cluster.map_shared_rank(my_x + cf + lc, p) = val;
         }
       }
       mma_phase ^= 1u;
       tc_fence_before_sync();
       __syncthreads();
-      issue(t + S - 1);
+      issue(t + S);  // into the slot just consumed
     }
 
-    // ---- exchange (t, eps) across the cluster; min/max of t, max of eps
+    // ---- all scores are local now; thread t owns candidates [t*PER, (t+1)*PER)
     if (C > 1) cluster.sync();
+    float tv[PER], ev[PER];
+    const int ibase = tid * PER;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int i = ibase + q;
+      const float2 x = i < ncand ? my_x[i] : make_float2(0.0f, 0.0f);
+      tv[q] = x.x;
+      ev[q] = x.y;
+    }
     float lo = INFINITY, hi = -INFINITY, emax = 0.0f;
-    {
-      float2 v[kMaxPer];
 #pragma unroll
-      for (int jj = 0; jj < kMaxPer; ++jj) {
-        const int i = tid + jj * kThreads;
-        v[jj] = make_float2(0.0f, 0.0f);
-        if (i < ncand) {
-          if (C > 1) {
-            const int peer = i / per_cta;
-            const float2* src = cluster.map_shared_rank(xch + buf * per_cta, peer);
-            v[jj] = src[i - peer * per_cta];
-          } else {
-            v[jj] = make_float2(sc_t[i], sc_e[i]);
-          }
-        }
-      }
-#pragma unroll
-      for (int jj = 0; jj < kMaxPer; ++jj) {
-        const int i = tid + jj * kThreads;
-        if (i < ncand) {
-          sc_t[i] = v[jj].x;
-          sc_e[i] = v[jj].y;
-          lo = fminf(lo, v[jj].x);
-          hi = fmaxf(hi, v[jj].x);
-          emax = fmaxf(emax, v[jj].y);
-        }
+    for (int q = 0; q < PER; ++q) {
+      if (ibase + q < ncand) {
+        if (tv[q] == 0.0f) tv[q] = 0.0f;  // -0 and +0 are the same score
+        lo = fminf(lo, tv[q]);
+        hi = fmaxf(hi, tv[q]);
+        emax = fmaxf(emax, ev[q]);
       }
     }
 #pragma unroll
@@ -384,6 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       fscratch[24 + warp] = hi;
       fscratch[32 + warp] = emax;
     }
+    if (tid == 0) {
+      uscratch[44] = 0u;           // band size
+      uscratch[45] = 0u;           // sure-in count
+      uscratch[46] = 0xffffffffu;  // min score key in the cut bucket
+      uscratch[47] = 0u;           // max score key in the cut bucket
+    }
     __syncthreads();
     lo = fscratch[16]; hi = fscratch[24]; emax = fscratch[32];
 #pragma unroll
@@ -393,59 +395,62 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       emax = fmaxf(emax, fscratch[32 + w]);
     }
 
-    // ---- theta = n0-th largest tensor-core score (bucket select)
+    // ---- the cut: bucket of the n0-th largest tensor-core score; buckets
+    // floor((t - lo) * scale) are non-decreasing in t
     const float scale = hi > lo ? static_cast<float>(kBuckets - 1) / (hi - lo) : 0.0f;
-    for (int i = tid; i < ncand; i += kThreads) {
-      int bi = static_cast<int>((sc_t[i] - lo) * scale);
-      bi = min(max(bi, 0), kBuckets - 1);
-      bkt[i] = static_cast<uint16_t>(bi);
-      atomicAdd(&hist[bi], 1);
+    int bv[PER];
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      bv[q] = min(max(static_cast<int>((tv[q] - lo) * scale), 0), kBuckets - 1);
+      if (ibase + q < ncand) atomicAdd(&hist[bv[q]], 1);
     }
     __syncthreads();
-    int cut, want;
-    find_cut(hist, n0, scratch, &cut, &want);
-    if (tid == 0) scratch[42] = 0;
-    __syncthreads();
-    for (int i = tid; i < ncand; i += kThreads)
-      if (bkt[i] == cut) mem[atomicAdd(&scratch[42], 1)] = i;
-    __syncthreads();
-    const int nmem = scratch[42];
-    for (int m = tid; m < nmem; m += kThreads) {
-      const int i = mem[m];
-      const float s = sc_t[i];
-      int r = 0;
-      for (int x = 0; x < nmem; ++x) {
-        const int jx = mem[x];
-        const float t2 = sc_t[jx];
-        r += (t2 > s || (t2 == s && jx < i)) ? 1 : 0;
+    const int cut = find_cut(hist, n0, scratch);
+    // the canonical n0-th largest score lies in [min_cut - emax, max_cut + emax]
+    uint32_t kmin = 0xffffffffu, kmaxv = 0u;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      if (ibase + q < ncand) {
+        if (bv[q] == cut) {
+          const uint32_t kq = score_key(tv[q]);
+          kmin = min(kmin, kq);
+          kmaxv = max(kmaxv, kq);
+        }
+        hist[bv[q]] = 0;  // ready for the next round
       }
-      if (r == want - 1) fscratch[43] = s;
     }
-    if (tid == 0) {
-      scratch[44] = 0;  // band size
-      scratch[45] = 0;  // sure-in count
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmaxv = max(kmaxv, __shfl_xor_sync(0xffffffffu, kmaxv, o));
     }
-    for (int i = tid; i < ncand; i += kThreads) hist[bkt[i]] = 0;  // for the next round
+    if (lane == 0) {
+      atomicMin(&uscratch[46], kmin);
+      atomicMax(&uscratch[47], kmaxv);
+    }
     __syncthreads();
-    const float theta = fscratch[43];
+    const float upper = key_score(uscratch[47]) + emax;  // >= canonical cut score
+    const float lower = key_score(uscratch[46]) - emax;  // <= canonical cut score
 
     // ---- classify: sure in (2), band (1), sure out (0)
+    uint8_t cl[PER];
     int nin = 0;
-    for (int i = tid; i < ncand; i += kThreads) {
-      const float t = sc_t[i], e = sc_e[i];
-      uint8_t c = 1;
-      if (t - e > theta + emax) c = 2;
-      else if (t + e < theta - emax) c = 0;
-      cls[i] = c;
-      nin += c == 2 ? 1 : 0;
-      if (c == 1) band[atomicAdd(&scratch[44], 1)] = i;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      cl[q] = 0;
+      if (ibase + q < ncand) {
+        const float t = tv[q], e = ev[q];
+        cl[q] = t - e > upper ? 2 : (t + e < lower ? 0 : 1);
+        nin += cl[q] == 2 ? 1 : 0;
+        if (cl[q] == 1) band[atomicAdd(&uscratch[44], 1u)] = ibase + q;
+      }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) nin += __shfl_xor_sync(0xffffffffu, nin, o);
-    if (lane == 0) atomicAdd(&scratch[45], nin);
+    if (lane == 0 && nin) atomicAdd(&uscratch[45], static_cast<uint32_t>(nin));
     __syncthreads();
-    const int nband = scratch[44];
-    const int need = n0 - scratch[45];
+    const int nband = static_cast<int>(uscratch[44]);
+    const int need = n0 - static_cast<int>(uscratch[45]);
     for (int m = tid; m < nband; m += kThreads) band_key[m] = 0u;
     __syncthreads();
 
@@ -460,18 +465,17 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         const int rem = live ? it - m * (bk * nrc) : 0;
         const int kt = rem / nrc, rc = rem - kt * nrc;
         const int ci = band[m];
-        const int64_t j = (cand_s[ci] + (cand_e[ci] - cand_s[ci]) / 2) * static_cast<int64_t>(bk) + kt;
+        const int64_t j = rep_key(ci) + kt;
         const bool jok = live && j < Tc;
         float kx[16];
         load_row16<uint16_t>(kbase + (jok ? j : 0) * 256, lane8, kx);
         float part[8];
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) {
-          const int r = rc * 8 + rr;
+          const int r = min(rc * 8 + rr, N - 1);
           float qv[16];
-          const int rq = r < N ? r : 0;
-          const uint4 x0 = *reinterpret_cast<const uint4*>(bq + sw128_offset(rq, lane8));
-          const uint4 x1 = *reinterpret_cast<const uint4*>(bq + N * 128 + sw128_offset(rq, lane8));
+          const uint4 x0 = *reinterpret_cast<const uint4*>(bq + sw128_offset(r, lane8));
+          const uint4 x1 = *reinterpret_cast<const uint4*>(bq + N * 128 + sw128_offset(r, lane8));
           qv[0] = bf16lo(x0.x); qv[1] = bf16hi(x0.x); qv[2] = bf16lo(x0.y); qv[3] = bf16hi(x0.y);
           qv[4] = bf16lo(x0.z); qv[5] = bf16hi(x0.z); qv[6] = bf16lo(x0.w); qv[7] = bf16hi(x0.w);
           qv[8] = bf16lo(x1.x); qv[9] = bf16hi(x1.x); qv[10] = bf16lo(x1.y); qv[11] = bf16hi(x1.y);
@@ -492,36 +496,64 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       }
     }
     __syncthreads();
-    // best `need` of the band by (canonical score desc, start asc)
-    for (int m = tid; m < nband; m += kThreads) {
+    // the band's best `need` by (canonical score desc, start asc): one warp per member
+    for (int m = warp; m < nband; m += kWarps) {
       const uint32_t km = band_key[m];
       const int im = band[m];
       int r = 0;
-      for (int x = 0; x < nband; ++x) {
+      for (int x = lane; x < nband; x += 32) {
         const uint32_t kx2 = band_key[x];
         r += (kx2 > km || (kx2 == km && band[x] < im)) ? 1 : 0;
       }
-      cls[im] = r < need ? 2 : 0;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+      if (lane == 0) keepb[im] = r < need ? 1 : 0;
     }
     __syncthreads();
 
-    // ---- order-preserving compaction of the kept candidates
-    const int per_c = (ncand + kThreads - 1) / kThreads;
-    const int lo_c = min(ncand, tid * per_c), hi_c = min(ncand, lo_c + per_c);
-    int nk = 0;
-    for (int i = lo_c; i < hi_c; ++i) nk += cls[i] == 2 ? 1 : 0;
-    int total;
-    int dst = block_excl_scan(nk, scratch, total);
-    for (int i = lo_c; i < hi_c; ++i) {
-      if (cls[i] == 2) {
-        chunk_s[dst] = cand_s[i];
-        chunk_e[dst] = cand_e[i];
-        ++dst;
+    // ---- keep and split: the kept candidates, in start order, become the
+    // next round's chunks; their halves (or themselves, when one block long)
+    // are written straight into the other candidate buffer
+    int cnt = 0, nl = 0;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int i = ibase + q;
+      if (i < ncand && (cl[q] == 2 || (cl[q] == 1 && keepb[i]))) {
+        const int len = ce[i] - cs[i];
+        cnt += len > 1 ? 2 : 1;
+        nl += len > 1 ? 1 : 0;
+      } else {
+        cl[q] = 0;
+      }
+      if (cl[q] == 1) cl[q] = 2;
+    }
+    int tot;
+    int pos = block_excl_scan(cnt | (nl << 16), scratch, tot) & 0xffff;
+    int* ns = cs_all + (cur ^ 1) * nbuf;
+    int* ne = ce_all + (cur ^ 1) * nbuf;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int i = ibase + q;
+      if (cl[q] == 2) {
+        const int s0 = cs[i], e0 = ce[i];
+        if (e0 - s0 > 1) {
+          const int m = s0 + (e0 - s0) / 2;
+          ns[pos] = s0; ne[pos] = m; ++pos;
+          ns[pos] = m; ne[pos] = e0; ++pos;
+        } else {
+          ns[pos] = s0; ne[pos] = e0; ++pos;
+        }
       }
     }
+    ncand = tot & 0xffff;
+    nlong = tot >> 16;
+    cur ^= 1;
+    if (C > 1) buf ^= 1;
     __syncthreads();
-    buf ^= 1;
   }
+  // every kept chunk is one block: the current candidate list (n0 entries,
+  // ascending) is the kept set
+  const int* chunk_s = cs_all + cur * nbuf;
 
   // ---- union with sink and window blocks, write the idx row (CTA 0)
   if (rank == 0) {
@@ -562,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   if (C > 1) cluster.sync();  // peers may still read this CTA's scores
 }
 
-template <int NC>
+template <int NC, int PER>
 cudaError_t prepare(const MaskArgs& a, int smem) {
   static int smem_set[kMaxDevices] = {};
   static bool big_cluster_set[kMaxDevices] = {};
@@ -571,19 +603,19 @@ cudaError_t prepare(const MaskArgs& a, int smem) {
   if (e != cudaSuccess) return e;
   dev %= kMaxDevices;
   if (smem > smem_set[dev]) {
-    e = cudaFuncSetAttribute(mask_mma_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(mask_mma_kernel<NC, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     smem_set[dev] = smem;
   }
   if (a.cluster > 8 && !big_cluster_set[dev]) {
-    e = cudaFuncSetAttribute(mask_mma_kernel<NC>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(mask_mma_kernel<NC, PER>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     big_cluster_set[dev] = true;
   }
   return cudaSuccess;
 }
 
-template <int NC>
+template <int NC, int PER>
 cudaLaunchConfig_t make_config(const MaskArgs& a, int smem, cudaStream_t stream,
                                cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
@@ -600,25 +632,25 @@ cudaLaunchConfig_t make_config(const MaskArgs& a, int smem, cudaStream_t stream,
   return cfg;
 }
 
-template <int NC>
+template <int NC, int PER>
 cudaError_t launch_nc(const MaskArgs& a, int smem, cudaStream_t stream) {
-  cudaError_t e = prepare<NC>(a, smem);
+  cudaError_t e = prepare<NC, PER>(a, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_config<NC>(a, smem, stream, attr);
-  return cudaLaunchKernelEx(&cfg, mask_mma_kernel<NC>, a);
+  cudaLaunchConfig_t cfg = make_config<NC, PER>(a, smem, stream, attr);
+  return cudaLaunchKernelEx(&cfg, mask_mma_kernel<NC, PER>, a);
 }
 
-template <int NC>
+template <int NC, int PER>
 int resident_nc(const MaskArgs& a, int smem) {
-  if (prepare<NC>(a, smem) != cudaSuccess) {
+  if (prepare<NC, PER>(a, smem) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
   }
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_config<NC>(a, smem, nullptr, attr);
+  cudaLaunchConfig_t cfg = make_config<NC, PER>(a, smem, nullptr, attr);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, mask_mma_kernel<NC>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, mask_mma_kernel<NC, PER>, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
   }
@@ -640,22 +672,22 @@ int mask_mma_tile_keys() { return kM; }
 
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem) {
   switch (mask_mma_nc(a.rows_max)) {
-    case 1: return resident_nc<1>(a, smem);
-    case 2: return resident_nc<2>(a, smem);
-    case 4: return resident_nc<4>(a, smem);
-    case 8: return resident_nc<8>(a, smem);
-    case 16: return resident_nc<16>(a, smem);
+    case 1: return a.n0max <= 1024 ? resident_nc<1, 8>(a, smem) : resident_nc<1, 16>(a, smem);
+    case 2: return a.n0max <= 1024 ? resident_nc<2, 8>(a, smem) : resident_nc<2, 16>(a, smem);
+    case 4: return a.n0max <= 1024 ? resident_nc<4, 8>(a, smem) : resident_nc<4, 16>(a, smem);
+    case 8: return a.n0max <= 1024 ? resident_nc<8, 8>(a, smem) : resident_nc<8, 16>(a, smem);
+    case 16: return a.n0max <= 1024 ? resident_nc<16, 8>(a, smem) : resident_nc<16, 16>(a, smem);
     default: return -1;
   }
 }
 
 cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream) {
   switch (mask_mma_nc(a.rows_max)) {
-    case 1: return launch_nc<1>(a, smem, stream);
-    case 2: return launch_nc<2>(a, smem, stream);
-    case 4: return launch_nc<4>(a, smem, stream);
-    case 8: return launch_nc<8>(a, smem, stream);
-    case 16: return launch_nc<16>(a, smem, stream);
+    case 1: return a.n0max <= 1024 ? launch_nc<1, 8>(a, smem, stream) : launch_nc<1, 16>(a, smem, stream);
+    case 2: return a.n0max <= 1024 ? launch_nc<2, 8>(a, smem, stream) : launch_nc<2, 16>(a, smem, stream);
+    case 4: return a.n0max <= 1024 ? launch_nc<4, 8>(a, smem, stream) : launch_nc<4, 16>(a, smem, stream);
+    case 8: return a.n0max <= 1024 ? launch_nc<8, 8>(a, smem, stream) : launch_nc<8, 16>(a, smem, stream);
+    case 16: return a.n0max <= 1024 ? launch_nc<16, 8>(a, smem, stream) : launch_nc<16, 16>(a, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -50,7 +50,9 @@ extern "C" int hip_sparse_attn_noalloc(const void* q, const void* k, const void*
   hips::AttnArgs a;
   int smem = 0;
   size_t need = 0;
-  int st = hips::plan_sparse_attn_own_scratch(q, k, v, idx, params, out, &a, &smem, &need);
+  bool tensor_core = false;
+  int st = hips::plan_sparse_attn_own_scratch(q, k, v, idx, params, out, &a, &smem, &need,
+                                              &tensor_core);
   if (st) return st;
   if (need > kScratchBytes) return HIPS_ERR_TOO_LARGE;
   void* base = nullptr;
@@ -64,5 +66,6 @@ extern "C" int hip_sparse_attn_noalloc(const void* q, const void* k, const void*
   a.status = static_cast<hips::Status*>(base);
   a.counters = reinterpret_cast<unsigned int*>(static_cast<unsigned char*>(base) + kCounterOffset);
   a.part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kStatusBytes);
-  return hips::record_cuda_error(hips::launch_attn_fma(a, smem, stream));
+  return hips::record_cuda_error(tensor_core ? hips::launch_attn_mma(a, smem, stream)
+                                             : hips::launch_attn_fma(a, smem, stream));
 }

@@ -91,3 +91,68 @@ def test_equal_keys_every_candidate_in_the_band():
     got = idx.cpu().numpy().reshape(-1)
     assert got[0] == topk // bk
     assert list(got[1:1 + got[0]]) == list(range(topk // bk))
+
+
+def _gpu_attention(w, x, idx_ref=None, dense=False):
+    """(gpu idx, gpu out on gpu idx, gpu out on the oracle idx) for a prefill workload."""
+    import torch
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    osh, bkw = pu.shapes(w)
+    q, k, v = pu.torch_inputs(x, w)
+    s = hb.Session(**bkw)
+    if dense:
+        out = s.dense_attn(q, k, v)
+        torch.cuda.synchronize()
+        s.check()
+        return None, out.float().cpu().numpy().reshape(-1, 128), None
+    idx = s.mask(q, k)
+    out = s.sparse_attn(q, k, v, idx)
+    out_ref_idx = None
+    if idx_ref is not None:
+        ri = torch.from_numpy(idx_ref).to("cuda").reshape(idx.shape).contiguous()
+        out_ref_idx = s.sparse_attn(q, k, v, ri).float().cpu().numpy().reshape(-1, 128)
+    torch.cuda.synchronize()
+    s.check()
+    return (idx.cpu().numpy().reshape(-1, idx.shape[-1]), out.float().cpu().numpy().reshape(-1, 128),
+            out_ref_idx)
+
+
+@pytest.mark.parametrize("w", SMALL[:3], ids=[w.name for w in SMALL[:3]])
+def test_small_prefill_attention_on_tensor_cores(w):
+    x = _inputs(w)
+    osh, _ = pu.shapes(w)
+    ref_idx, gap, _ = oracle.mask(x["q"][0], x["k"], osh)
+    got_idx, out_e2e, out_on_ref = _gpu_attention(w, x, ref_idx)
+    ref = oracle.attention(x["q"][0], x["k"], x["v"], ref_idx, osh)
+    pu.compare_outputs(out_on_ref, ref, w.dtype)
+    st = pu.compare_masks(got_idx, ref_idx, gap)
+    if st["mismatched"] == 0:
+        pu.compare_outputs(out_e2e, ref, w.dtype)
+
+
+def test_small_prefill_dense_attention():
+    w = W.Workload("pd", "prefill", 1, 4, 2, 128, 1500, 64, 2, 256, 0, 0, "bf16")
+    x = _inputs(w)
+    osh, _ = pu.shapes(w)
+    _, out, _ = _gpu_attention(w, x, dense=True)
+    ref = oracle.attention(x["q"][0], x["k"], x["v"], None, osh)
+    pu.compare_outputs(out, ref, w.dtype)
+
+
+def test_prefill_32k_attention_sampled():
+    w = W.PREFILL_32K
+    x = _inputs(w)
+    osh, _ = pu.shapes(w)
+    got_idx, out, _ = _gpu_attention(w, x)
+    nqb = oracle.num_qblocks(osh)
+    G, bq, T = w.group, w.block_q, w.seq_len
+    picks = [(0, 0), (3, 31), (5, 32), (7, 33), (2, 200), (6, nqb - 1), (1, 400)]
+    units = np.array([g * nqb + qb for g, qb in picks], dtype=np.int64)
+    ref_idx, gap, _ = oracle.mask(x["q"][0], x["k"], osh, units=units)
+    pu.compare_masks(got_idx[units], ref_idx, gap)
+    full_idx = np.full((got_idx.shape[0], got_idx.shape[1]), -1, np.int32)
+    full_idx[units] = ref_idx
+    rows = np.array([(g * G + h) * T + qb * bq + i for g, qb in picks for h in range(G)
+                     for i in range(0, bq, 7)], dtype=np.int64)
+    ref = oracle.attention(x["q"][0], x["k"], x["v"], full_idx, osh, rows=rows)
+    pu.compare_outputs(out[rows], ref, w.dtype)
