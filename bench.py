@@ -78,30 +78,40 @@ def layer_shape(w: W.Workload):
                 kv_capacity=w.capacity)
 
 
-def mask_algorithmic_bytes(w: W.Workload) -> int:
+def mask_algorithmic_bytes(w: W.Workload, scored: int) -> int:
     """Bytes the mask must read: every round reads the representative key block
-    of each candidate (b_k keys x d), plus q; it writes the idx rows.
-
-    Exact for decode workloads, where every chunk has the same length in
-    every round (N / n0 is a power of two), so the candidate count is 2 n0."""
+    (b_k keys x d) of each candidate chunk, plus q; it writes the idx rows.
+    ``scored`` is the number of candidates the kernels scored in one call
+    (each candidate of each round exactly once)."""
     esz = 2 if w.dtype == "bf16" else 4
-    assert w.kind == "decode"
-    T, bk = w.seq_len, w.block_k
-    N = -(-T // bk)
-    n0 = min(w.topk // bk, N)
-    lens = [(i + 1) * N // n0 - i * N // n0 for i in range(n0)]
-    keys = 0
-    # all chunks equal: halve until single blocks, 2 n0 candidates per round
-    assert len(set(lens)) == 1
-    L = lens[0]
-    while L > 1:
-        keys += 2 * n0 * bk
-        L //= 2
-    units = w.batch * w.n_kvheads
-    stride = 1 + w.topk // bk + -(-w.sink // bk) + ((-(-(w.window + w.block_q - 1) // bk) + 1)
-                                                   if w.window else 0)
+    units = w.batch * w.n_kvheads * (-(-w.q_len // w.block_q))
+    stride = 1 + w.topk // w.block_k + -(-w.sink // w.block_k) + (
+        (-(-(w.window + w.block_q - 1) // w.block_k) + 1) if w.window else 0)
     q_bytes = w.batch * w.n_qheads * w.q_len * w.head_dim * esz
-    return units * keys * w.head_dim * esz + q_bytes + units * stride * 4
+    return scored * w.block_k * w.head_dim * esz + q_bytes + units * stride * 4
+
+
+def mask_algorithmic_flops(w: W.Workload, scored: int) -> int:
+    """Multiply-adds of the mask scores: every candidate's b_k keys against the
+    G * b_q query rows of its mask (d = 128), two flops each."""
+    return 2 * scored * w.block_k * w.group * w.block_q * w.head_dim
+
+
+def attn_algorithmic_flops(w: W.Workload, idx: np.ndarray) -> int:
+    """QK^T and PV flops (4 d per attended (row, key) pair), counted from the
+    idx rows: a row at position p attends the listed keys j <= p."""
+    bk, bq, T, G = w.block_k, w.block_q, w.seq_len, w.group
+    rows = idx.reshape(-1, idx.shape[-1])
+    nqb = rows.shape[0] // (w.batch * w.n_kvheads)
+    pairs = 0
+    for u, r in enumerate(rows):
+        qb = u % nqb
+        blocks = r[1:1 + r[0]].astype(np.int64)
+        keys = (blocks[:, None] * bk + np.arange(bk)[None, :]).reshape(-1)
+        keys = np.sort(keys[keys < T])
+        pos = np.arange(qb * bq, min(qb * bq + bq, w.q_len))
+        pairs += G * int(np.searchsorted(keys, pos, side="right").sum())
+    return 4 * w.head_dim * pairs
 
 
 def attn_algorithmic_bytes(w: W.Workload, idx: np.ndarray, seq_len: int, mask_len: int) -> int:
@@ -230,48 +240,66 @@ def max_over_ranks(x: float, world: int) -> float:
 
 def reference_arm(args, w: W.Workload, world: int, rank: int):
     """The CPU oracle, as it stands, on the host cores: each step runs the mask
-    and attention of a sample of the layer's KV-head units."""
+    and attention of a sample of the layer's (sequence, KV head, query block)
+    units, sized so that the whole run stays within a few minutes, and the
+    time is scaled to one layer. Same metric and unit as the GPU arm."""
     if rank != 0:
         return
     import oracle
     cores = oracle.set_threads(0)
     x = W.make_inputs(w)
     sh = oracle.shape(head_dim=w.head_dim, **layer_shape(w))
-    units = w.batch * w.n_kvheads * (-(-w.q_len // w.block_q))
-    G = w.group
-
-    def step(u: int, pick: np.ndarray):
-        idx, _, _ = oracle.mask(x["q"][0], x["k"], sh, units=pick)
-        full = np.full((units, idx.shape[1]), -1, np.int32)
-        full[pick] = idx
-        rows = np.concatenate([np.arange(p * G, (p + 1) * G) for p in pick])
-        oracle.attention(x["q"][0], x["k"], x["v"], full, sh, rows=rows)
-
+    nqb = -(-w.q_len // w.block_q)
+    units = w.batch * w.n_kvheads * nqb
+    prefill = w.kind == "prefill"
     rng = np.random.default_rng(0)
+    # calibrate on a spread sample (a whole prefill layer would take hours)
+    cal = np.unique(np.linspace(0, units - 1, min(units, max(cores, 8))).astype(np.int64))
     t0 = time.perf_counter()
-    step(units, np.arange(units))
-    t_layer = time.perf_counter() - t0
+    _oracle_units(w, x, sh, cal)
+    t_layer = (time.perf_counter() - t0) * units / cal.size
     budget = 150.0
     u = units
     while u > 1 and (args.steps + args.warmup) * t_layer * u / units > budget:
         u //= 2
-    for _ in range(max(0, args.warmup - 1)):
-        step(u, rng.choice(units, u, replace=False))
+    picks = [rng.choice(units, u, replace=False) for _ in range(args.steps + max(0, args.warmup - 1))]
+    for pick in picks[args.steps:]:
+        _oracle_units(w, x, sh, pick)
+    flops = 0
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step(u, rng.choice(units, u, replace=False))
+    for pick in picks[:args.steps]:
+        _oracle_units(w, x, sh, pick)
     elapsed = time.perf_counter() - t0
     us_layer = elapsed / args.steps * (units / u) * 1e6
-    sample = (f"{u} of {units} (sequence, KV head) units per step: their mask rows and the "
-              f"attention of their {G} query heads; scaled to one layer")
-    line = {"metric": METRIC, "value": us_layer, "unit": "us/layer", "impl": "reference",
+    sample = (f"{u} of {units} (sequence, KV head, query block) units per step: their mask rows "
+              f"and the attention of their query rows; scaled to one layer")
+    value, unit, hib = us_layer, "us/layer", False
+    if prefill:
+        # the flops of the sampled units (same count as the GPU arm), per second
+        for pick in picks[:1]:
+            idx, _, _, scored = oracle.mask(x["q"][0], x["k"], sh, units=pick, with_scored=True)
+            full = np.full((units, idx.shape[1]), -1, np.int32)
+            full[pick] = idx
+            sub = full[np.sort(pick)]
+            flops = mask_algorithmic_flops(w, int(scored.sum()))
+            for uu in np.sort(pick):
+                qb = uu % nqb
+                r = full[uu]
+                blocks = r[1:1 + r[0]].astype(np.int64)
+                keys = np.sort(((blocks[:, None] * w.block_k + np.arange(w.block_k)[None, :])
+                                .reshape(-1)))
+                pos = np.arange(qb * w.block_q, min(qb * w.block_q + w.block_q, w.q_len))
+                flops += 4 * w.head_dim * w.group * int(np.searchsorted(keys, pos, side="right").sum())
+            del sub
+        value, unit, hib = flops / (elapsed / args.steps) / 1e12, "TFLOP/s", True
+    line = {"metric": METRIC, "value": value, "unit": unit, "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": False,
+            "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": hib,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_of(w, 0),
-            "cpu_baseline": {"value": us_layer, "unit": "us/layer", "cores": cores,
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores,
                              "kind": "oracle", "sample": sample},
-            "e2e": {"value": us_layer, "unit": "us/layer", "h2d_bytes_per_step": 0,
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -284,11 +312,40 @@ def config_of(w: W.Workload, layers: int):
             "l2": f"{layers} rotating layer buffers > L2 (no flush)" if layers else None}
 
 
+def _oracle_units(w: W.Workload, x: dict, sh, units: np.ndarray):
+    """Oracle mask + attention of the given (sequence, KV head, query block) units."""
+    import oracle
+    nqb = -(-w.q_len // w.block_q)
+    idx, _, _ = oracle.mask(x["q"][0], x["k"], sh, units=units)
+    full = np.full((w.batch * w.n_kvheads * nqb, idx.shape[1]), -1, np.int32)
+    full[units] = idx
+    rows = []
+    for u in units:
+        qb, g, b = u % nqb, (u // nqb) % w.n_kvheads, u // (nqb * w.n_kvheads)
+        for h in range(g * w.group, (g + 1) * w.group):
+            base = (b * w.n_qheads + h) * w.q_len
+            rows.extend(range(base + qb * w.block_q, base + min(qb * w.block_q + w.block_q, w.q_len)))
+    oracle.attention(x["q"][0], x["k"], x["v"], full, sh, rows=np.asarray(rows, np.int64))
+
+
 def cpu_baseline(w: W.Workload, x: dict, min_seconds: float = 10.0):
-    """The oracle timed on whole layers of the workload until min_seconds pass."""
+    """The oracle timed on the host cores: whole layers (decode) until
+    min_seconds pass, or a spread sample of query blocks scaled to a layer
+    (prefill, where a whole layer takes hours)."""
     import oracle
     cores = oracle.set_threads(0)
     sh = oracle.shape(head_dim=w.head_dim, **layer_shape(w))
+    if w.kind == "prefill":
+        nqb = -(-w.q_len // w.block_q)
+        units_total = w.batch * w.n_kvheads * nqb
+        pick = np.unique(np.linspace(0, units_total - 1, max(cores, 8)).astype(np.int64))
+        t0 = time.perf_counter()
+        _oracle_units(w, x, sh, pick)
+        el = time.perf_counter() - t0
+        per_layer = el * units_total / pick.size
+        return {"value": per_layer * 1e6, "unit": "us/layer", "cores": cores, "kind": "oracle",
+                "sample": f"{pick.size} of {units_total} query blocks spread over the layer "
+                          f"(mask + attention), extrapolated linearly to the layer"}
     n = 0
     t0 = time.perf_counter()
     while True:
@@ -328,12 +385,11 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     from hierarchically_pruned_sparse_b200 import binding as hb
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if w.kind != "decode":
-        raise SystemExit(f"workload {w.name}: prefill benchmark not available yet")
     x = W.make_inputs(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     esz = 2 if w.dtype == "bf16" else 4
-    layer_bytes = 2 * x["k"].size * esz
+    prefill = w.kind == "prefill"
+    layer_bytes = (2 * x["k"].size + x["q"][0].size) * esz
     layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
     layers = min(layers, 64)
     k0 = torch.from_numpy(x["k"]).to(dev).to(dt).contiguous()
@@ -358,9 +414,19 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
             step(i % layers)
     stream.synchronize()
     sess.check()
+    # one more mask call on a cleared status block counts the scored candidates
+    hb.workspace_init(sess.p)
+    with torch.cuda.stream(stream):
+        hb.hip_mask(qs[0], ks[0], sess.p, idxs[0])
+    stream.synchronize()
+    base = sess.p.workspace - sess.workspace.data_ptr()
+    scored = int(sess.workspace[base + 8: base + 16].cpu().numpy().view(np.uint64)[0])
+    sess.check()
     idx_host = idxs[0].cpu().numpy()
-    mask_bytes = mask_algorithmic_bytes(w)
+    mask_bytes = mask_algorithmic_bytes(w, scored)
     attn_bytes = attn_algorithmic_bytes(w, idx_host, w.seq_len, w.seq_len)
+    mask_flops = mask_algorithmic_flops(w, scored)
+    attn_flops = attn_algorithmic_flops(w, idx_host) if prefill else 0
 
     # CUDA graphs of `layers` steps (and of the remainder of K), with
     # per-kernel events in the full graph
@@ -407,15 +473,19 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     us_layer = total_ms * 1e3 / (steps * world)
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
+    tensor_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
     mask_gbs = mask_bytes / (mask_ms * 1e-3) / 1e9
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
     step_gbs = (mask_bytes + attn_bytes) / (total_ms * 1e-3 / (steps)) / 1e9
+    mask_tf = mask_flops / (mask_ms * 1e-3) / 1e12
+    attn_tf = attn_flops / (attn_ms * 1e-3) / 1e12
+    step_tf = (mask_flops + attn_flops) / (total_ms * 1e-3 / steps) / 1e12
     launches_per_step = 2  # hip_mask + hip_sparse_attn (the split merge is fused)
 
     # e2e: per step, H2D of the step's query and new key/value rows from pinned
     # host memory, the two C-ABI calls, D2H of the output; captured as a graph
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not prefill:
         hq = [torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dt).pin_memory() for _ in range(layers)]
         krow = torch.from_numpy(np.ascontiguousarray(x["k"][:, :, w.seq_len - 1])).to(dt).pin_memory()
         vrow = torch.from_numpy(np.ascontiguousarray(x["v"][:, :, w.seq_len - 1])).to(dt).pin_memory()
@@ -458,29 +528,78 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
                "how": "CUDA graph of H2D (pinned) + hip_mask + hip_sparse_attn + D2H per step"}
         sess.check()
 
+    if not args.no_e2e and prefill:
+        hq = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dt).pin_memory()
+        hk = torch.from_numpy(x["k"]).to(dt).pin_memory()
+        hv = torch.from_numpy(x["v"]).to(dt).pin_memory()
+        hout = torch.empty(q0.shape, dtype=dt).pin_memory()
+        n_e2e = max(1, min(steps, 20))
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            s2.record(stream)
+            for i in range(n_e2e):
+                l = i % layers
+                qs[l].copy_(hq, non_blocking=True)
+                ks[l].copy_(hk, non_blocking=True)
+                vs[l].copy_(hv, non_blocking=True)
+                step(l)
+                hout.copy_(outs[l], non_blocking=True)
+            e2.record(stream)
+        e2.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2), world)
+        fl = (mask_flops + attn_flops) * n_e2e * world
+        e2e = {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int((hq.numel() + hk.numel() + hv.numel()) * esz),
+               "d2h_bytes_per_step": int(q0.numel() * esz), "steps": n_e2e,
+               "how": "per step: H2D of q, k, v (pinned), hip_mask, hip_sparse_attn, D2H of out"}
+        sess.check()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, x)
 
-    traffic = traffic_from_profile("mask_fma_kernel", w.name)
+    mask_kernel = "mask_mma_kernel" if w.dtype == "bf16" else "mask_fma_kernel"
+    attn_kernel = "attn_mma_kernel" if prefill else "attn_fma_kernel"
+    if prefill:
+        dom_attn = attn_ms >= mask_ms
+        dom_tf = attn_tf if dom_attn else mask_tf
+        roofline = {"bound": "tensor", "kernel": attn_kernel if dom_attn else mask_kernel,
+                    "achieved": dom_tf, "peak": tensor_peak, "peak_kind": f"{pk_kind} bf16 sustained",
+                    "unit": "TFLOP/s", "frac": dom_tf / tensor_peak,
+                    "traffic": traffic_from_profile(attn_kernel if dom_attn else mask_kernel, w.name),
+                    "algorithmic_flops": attn_flops if dom_attn else mask_flops}
+        value, unit, hib = step_tf, "TFLOP/s", True
+    else:
+        roofline = {"bound": "hbm", "kernel": mask_kernel, "achieved": mask_gbs,
+                    "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s", "frac": mask_gbs / hbm,
+                    "traffic": traffic_from_profile(mask_kernel, w.name),
+                    "algorithmic_bytes": mask_bytes}
+        value, unit, hib = us_layer, "us/layer", False
     line = {
-        "metric": METRIC, "value": us_layer, "unit": "us/layer", "n_gpus": world,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
         "steps": steps, "warmup": args.warmup, "ms_per_step": total_ms / steps,
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": hib, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if dt == torch.bfloat16 else "f32",
         "data": "synthetic (seeded AR(1) keys/values, Gaussian queries, needle keys)",
         "config": config_of(w, layers),
-        "roofline": {"bound": "hbm", "kernel": "mask_fma_kernel", "achieved": mask_gbs,
-                     "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s", "frac": mask_gbs / hbm,
-                     "traffic": traffic, "algorithmic_bytes": mask_bytes},
+        "roofline": roofline,
         "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": step_gbs / hbm, "algorithmic_bytes": mask_bytes + attn_bytes},
         "kernels": {"how": "CUDA event nodes around each call, last full graph replay of the timed region",
+                    "mask_kernel": mask_kernel, "attn_kernel": attn_kernel,
                     "mask_us": mask_ms * 1e3, "mask_bytes": mask_bytes, "mask_gbs": mask_gbs,
-                    "attn_us": attn_ms * 1e3, "attn_bytes": attn_bytes, "attn_gbs": attn_gbs},
+                    "mask_tflops": mask_tf, "mask_flops": mask_flops, "scored_candidates": scored,
+                    "attn_us": attn_ms * 1e3, "attn_bytes": attn_bytes, "attn_gbs": attn_gbs,
+                    "attn_tflops": attn_tf, "attn_flops": attn_flops},
         "gpu_launches": launches_per_step * steps,
         "clocks": clk.summary(),
     }
+    if prefill:
+        line["step_tflops"] = step_tf
+        line["us_per_layer"] = us_layer
     if e2e:
         line["e2e"] = e2e
     if cpu:

@@ -14,10 +14,13 @@ constexpr int kMaxDevices = 64;
 constexpr unsigned kStatusTimeout = 1u;
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 
-// Status block at the head of every workspace (sticky error bits).
+// Status block at the head of every workspace (sticky error bits), plus the
+// number of candidate chunks the mask kernels scored since the block was
+// cleared (a work counter: every candidate is scored exactly once).
 struct Status {
   unsigned int flags;
   unsigned int where;
+  unsigned long long scored;
 };
 
 __device__ __forceinline__ void report(Status* st, unsigned bits, unsigned where) {

@@ -295,6 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
     }
     seq += static_cast<uint32_t>(ntiles);
 
+    if (tid == 0 && a.status && c_hi > c_lo)
+      atomicAdd(&a.status->scored, static_cast<unsigned long long>(c_hi - c_lo));
     // ---- exchange scores across the cluster (batched DSMEM loads); track min/max
     if (C > 1) cluster.sync();
     float lo = INFINITY, hi = -INFINITY;

@@ -348,6 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       issue(t + S);  // into the slot just consumed
     }
 
+    if (tid == 0 && a.status && c_hi > c_lo)
+      atomicAdd(&a.status->scored, static_cast<unsigned long long>(c_hi - c_lo));
     // ---- all scores are local now; thread t owns candidates [t*PER, (t+1)*PER)
     if (C > 1) cluster.sync();
     float tv[PER], ev[PER];

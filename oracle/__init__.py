@@ -73,7 +73,7 @@ def _load():
     lib.oracle_set_threads.restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_mask.restype = ctypes.c_int
-    lib.oracle_mask.argtypes = [f32p, f32p, P(Shape), i64p, ctypes.c_int64, i32p, f64p, i32p]
+    lib.oracle_mask.argtypes = [f32p, f32p, P(Shape), i64p, ctypes.c_int64, i32p, f64p, i32p, i64p]
     lib.oracle_attention.restype = ctypes.c_int
     lib.oracle_attention.argtypes = [f32p, f32p, f32p, i32p, P(Shape), i64p, ctypes.c_int64, f32p]
     _lib = lib
@@ -117,13 +117,14 @@ def num_qblocks(sh: Shape) -> int:
     return int(_load().oracle_num_qblocks(ctypes.byref(sh)))
 
 
-def mask(q, k, sh: Shape, units=None):
+def mask(q, k, sh: Shape, units=None, with_scored=False):
     """Hierarchical top-k masks.
 
     q: [B, Hq, Lq, d]; k: [B, Hkv, kv_capacity, d] (float32 values).
     Returns (idx [n_units, 1 + cap] int32, gap [n_units] float64,
-    rounds [n_units] int32), units in (b, g, qb) row-major order unless an
-    explicit list of flattened unit ids is given.
+    rounds [n_units] int32) -- plus scored [n_units] int64, the candidates
+    scored over all rounds, when with_scored -- units in (b, g, qb) row-major
+    order unless an explicit list of flattened unit ids is given.
     """
     lib = _load()
     q, k = _f32(q), _f32(k)
@@ -133,12 +134,15 @@ def mask(q, k, sh: Shape, units=None):
     idx = np.empty((n, 1 + idx_cap(sh)), dtype=np.int32)
     gap = np.empty(n, dtype=np.float64)
     rounds = np.empty(n, dtype=np.int32)
+    scored = np.empty(n, dtype=np.int64)
     st = lib.oracle_mask(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float), ctypes.byref(sh),
                          None if u is None else _ptr(u, ctypes.c_int64), n,
                          _ptr(idx, ctypes.c_int32), _ptr(gap, ctypes.c_double),
-                         _ptr(rounds, ctypes.c_int32))
+                         _ptr(rounds, ctypes.c_int32), _ptr(scored, ctypes.c_int64))
     if st != 0:
         raise RuntimeError(f"oracle_mask failed ({st})")
+    if with_scored:
+        return idx, gap, rounds, scored
     return idx, gap, rounds
 
 

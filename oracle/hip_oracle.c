@@ -133,7 +133,7 @@ static int cand_order(const void* pa, const void* pb) {
  * then the sink/window union of [Summary] and the idx+nnz row of [NLBm] W2).
  */
 static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int64_t unit,
-                     int32_t* row, double* gap_out, int32_t* rounds_out) {
+                     int32_t* row, double* gap_out, int32_t* rounds_out, int64_t* scored_out) {
   const int d = sh->head_dim, G = sh->n_qheads / sh->n_kvheads;
   const int64_t nqb = oracle_num_qblocks(sh), bk = sh->block_k;
   const int64_t qb = unit % nqb, g = (unit / nqb) % sh->n_kvheads, b = unit / (nqb * sh->n_kvheads);
@@ -156,6 +156,7 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
   }
   double gap = INFINITY;
   int32_t rounds = 0;
+  int64_t scored = 0;
   for (;;) {
     int64_t nc = 0, longest = 0;
     for (int64_t i = 0; i < n0; ++i) longest = max64(longest, chunks[i].e - chunks[i].s);
@@ -172,6 +173,7 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
       }
     }
     /* step 3: score each half by its centre block */
+    scored += nc;
     for (int64_t c = 0; c < nc; ++c) {
       int64_t rep = cands[c].s + (cands[c].e - cands[c].s) / 2;
       float best = -INFINITY;
@@ -213,6 +215,7 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
   for (int64_t i = nnz; i < cap; ++i) row[1 + i] = -1;
   if (gap_out) *gap_out = gap;
   if (rounds_out) *rounds_out = rounds;
+  if (scored_out) *scored_out = scored;
   free(chunks); free(cands); free(keep);
   return nnz <= cap ? OR_OK : OR_BAD;
 }
@@ -222,10 +225,12 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
  * units when units == NULL. idx_out holds one row of 1 + cap int32 per unit:
  * [nnz, ascending block ids..., -1 padding]. gap_out (optional) gets the
  * smallest score gap at the cut over the rounds, in q.k/sqrt(d) units
- * (+inf when no round had more candidates than survivors).
+ * (+inf when no round had more candidates than survivors). rounds_out and
+ * scored_out (optional) count the rounds and the candidates scored.
  */
 int oracle_mask(const float* q, const float* k, const oracle_shape* sh, const int64_t* units,
-                int64_t n_units, int32_t* idx_out, double* gap_out, int32_t* rounds_out) {
+                int64_t n_units, int32_t* idx_out, double* gap_out, int32_t* rounds_out,
+                int64_t* scored_out) {
   if (!q || !k || !idx_out || !shape_ok(sh)) return OR_BAD;
   const int64_t total = (int64_t)sh->batch * sh->n_kvheads * oracle_num_qblocks(sh);
   if (!units) n_units = total;
@@ -236,7 +241,7 @@ int oracle_mask(const float* q, const float* k, const oracle_shape* sh, const in
     int64_t unit = units ? units[u] : u;
     int st = (unit < 0 || unit >= total) ? OR_BAD
              : mask_unit(q, k, sh, unit, idx_out + u * stride, gap_out ? gap_out + u : NULL,
-                         rounds_out ? rounds_out + u : NULL);
+                         rounds_out ? rounds_out + u : NULL, scored_out ? scored_out + u : NULL);
     if (st != OR_OK) {
 #pragma omp critical
       status = st;

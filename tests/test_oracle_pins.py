@@ -347,3 +347,18 @@ def test_sink_and_window_blocks_always_present():
     want = set(idx0[0, 1:1 + idx0[0, 0]]) | set(range(64)) | set(range((T - 1024) // 2, T // 2))
     assert got == want
     assert idx[0, 0] <= oracle.idx_cap(sh)
+
+
+@pytest.mark.parametrize("T,bk,topk", [(8192, 16, 512), (131072, 2, 2048), (4096, 4, 256)])
+def test_scored_candidates_closed_form(T, bk, topk):
+    # equal-length chunks: every round scores exactly 2 n0 candidates
+    rng = np.random.default_rng(1)
+    d = 128
+    q = rng.standard_normal((1, 2, 1, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    sh = _shape(batch=1, n_qheads=2, n_kvheads=1, head_dim=d, seq_len=T, q_len=1, q_pos0=T - 1,
+                block_q=1, block_k=bk, topk=topk)
+    _, _, rounds, scored = oracle.mask(q, k, sh, with_scored=True)
+    n0 = topk // bk
+    assert rounds[0] == int(math.log2((T // bk) // n0))
+    assert scored[0] == 2 * n0 * rounds[0]
