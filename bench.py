@@ -447,15 +447,17 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         with torch.cuda.graph(g_rem, stream=stream):
             for l in range(rem):
                 step(l)
-    for _ in range(2):
-        g.replay()
-        if g_rem is not None:
-            g_rem.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g.replay()
+            if g_rem is not None:
+                g_rem.replay()
     stream.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):
+        # graphs replay on the current stream: make it the stream the events use
         start.record(stream)
         for _ in range(reps):
             g.replay()
@@ -508,17 +510,19 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
             with torch.cuda.graph(g2_rem, stream=stream):
                 for l in range(rem):
                     e2e_step(l)
-        g2.replay()
+        with torch.cuda.stream(stream):
+            g2.replay()
         stream.synchronize()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize(dev)
-        s2.record(stream)
-        for _ in range(reps):
-            g2.replay()
-        if g2_rem is not None:
-            g2_rem.replay()
-        e2.record(stream)
+        with torch.cuda.stream(stream):
+            s2.record(stream)
+            for _ in range(reps):
+                g2.replay()
+            if g2_rem is not None:
+                g2_rem.replay()
+            e2.record(stream)
         e2.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), world)

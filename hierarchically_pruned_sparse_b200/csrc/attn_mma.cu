@@ -82,8 +82,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   const int R = a.group * nrows;
   const int64_t q_first = a.q_pos0 + i0, q_last = q_first + nrows - 1;
   const int64_t vis = min64(q_last + 1, a.seq_len);
-  const int IK = a.item_keys;
-  const int ipt = kKeys / IK;
+  const int IK = a.item_keys;  // a power of two
+  const int lik = __ffs(IK) - 1;
+  const int ipt = kKeys >> lik;
   const int row0 = mt * kRows;
 
   const AttnMmaSmem L = attn_mma_layout(a.table_items);
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
       for (int m = 0; m < (kKeys * 16) / 128; ++m) {
         const int i = lt + 128 * m;
         const int kk = i >> 4, ch = i & 15;
-        const int item = j * ipt + kk / IK, kt = kk % IK;
+        const int item = j * ipt + (kk >> lik), kt = kk & (IK - 1);
         if (item < nitems) {
           const int2 e = table[item];
           if (kt < e.y) {
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
       if (tid < kKeys) {
-        const int item = j * ipt + tid / IK, kt = tid % IK;
+        const int item = j * ipt + (tid >> lik), kt = tid & (IK - 1);
         int kp = -1;
         if (item < nitems) {
           const int2 e = table[item];
@@ -313,10 +314,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 w;
-        w.x = static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 0])) | (static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 1])) << 16);
-        w.y = static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 2])) | (static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 3])) << 16);
-        w.z = static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 4])) | (static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 5])) << 16);
-        w.w = static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 6])) | (static_cast<uint32_t>(f2bf16_rn(p[c * 8 + 7])) << 16);
+        w.x = pack_bf16x2(p[c * 8 + 0], p[c * 8 + 1]);
+        w.y = pack_bf16x2(p[c * 8 + 2], p[c * 8 + 3]);
+        w.z = pack_bf16x2(p[c * 8 + 4], p[c * 8 + 5]);
+        w.w = pack_bf16x2(p[c * 8 + 6], p[c * 8 + 7]);
         *reinterpret_cast<uint4*>(prow + sw128_offset(tid, c)) = w;
       }
       fence_proxy_async_smem();
@@ -351,10 +352,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         uint32_t* u1 = &w1.x;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          u0[i] = static_cast<uint32_t>(f2bf16_rn(v[2 * i] * inv)) |
-                  (static_cast<uint32_t>(f2bf16_rn(v[2 * i + 1] * inv)) << 16);
-          u1[i] = static_cast<uint32_t>(f2bf16_rn(v[8 + 2 * i] * inv)) |
-                  (static_cast<uint32_t>(f2bf16_rn(v[8 + 2 * i + 1] * inv)) << 16);
+          u0[i] = pack_bf16x2(v[2 * i] * inv, v[2 * i + 1] * inv);
+          u1[i] = pack_bf16x2(v[8 + 2 * i] * inv, v[8 + 2 * i + 1] * inv);
         }
         *reinterpret_cast<uint4*>(orow + c * 16) = w0;
         *reinterpret_cast<uint4*>(orow + c * 16 + 8) = w1;

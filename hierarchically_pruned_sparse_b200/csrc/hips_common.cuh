@@ -113,6 +113,13 @@ __device__ __forceinline__ uint16_t f2bf16_rn(float f) {
   return static_cast<uint16_t>(u >> 16);
 }
 
+// Two floats to packed bf16x2 (round to nearest even); lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Order-preserving map of a float score onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t score_key(float f) {
   if (f == 0.0f) f = 0.0f;  // -0 and +0 are the same score

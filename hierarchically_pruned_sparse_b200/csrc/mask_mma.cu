@@ -51,7 +51,7 @@ __host__ __device__ constexpr int stages_for(int nc) { return nc >= 16 ? 2 : nc 
 __host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 16 < 32 ? 32 : nc * 16; }
 
 struct MmaSmem {
-  int ring, bq, bar, slot, cs, ce, keepb, band, band_key, xch, hist, scratch, total;
+  int ring, bq, bar, slot, rpos, cs, ce, keepb, band, band_key, xch, hist, scratch, total;
 };
 
 __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
@@ -68,6 +68,7 @@ __host__ __device__ inline MmaSmem mma_layout(int nc, int n0max, int per_cta, in
   L.bq = o;       o += nc * 16 * 256;
   L.bar = o;      o += 16;
   L.slot = o;     o += 16;
+  L.rpos = o;     o += nc * 16 * 4;  // query position offset (r % b_q) of operand row r
   L.cs = o;       o += 2 * al(n * 4, 16);
   L.ce = o;       o += 2 * al(n * 4, 16);
   L.keepb = o;    o += al(n, 16);
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   unsigned char* bq = smem + L.bq;
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.slot);
+  int* rpos = reinterpret_cast<int*>(smem + L.rpos);
   int* cs_all = reinterpret_cast<int*>(smem + L.cs);
   int* ce_all = reinterpret_cast<int*>(smem + L.ce);
   uint8_t* keepb = reinterpret_cast<uint8_t*>(smem + L.keepb);
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     *reinterpret_cast<uint4*>(bq + (c >> 3) * (N * 128) + sw128_offset(r, c & 7)) = v;
   }
   for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
+  for (int r = tid; r < N; r += kThreads) rpos[r] = r < R ? r % nrows : -1;  // -1: padding row
 
   // ---- candidates of round 1: the halves of the n0 initial chunks
   // (a one-block chunk stays whole); thread t owns chunks [t*pc, (t+1)*pc)
@@ -318,15 +321,25 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         __syncwarp();
         float tsc = -INFINITY;
         const bool full = j <= q_first;  // every row sees this key
+        const int64_t jrel = j - q_first;   // otherwise row r needs r % b_q >= jrel
+        constexpr int kBatch = NC < 4 ? NC : 4;
+#pragma unroll 1
+        for (int ch0 = 0; ch0 < NC; ch0 += kBatch) {
+          float v[kBatch][16];
 #pragma unroll
-        for (int ch = 0; ch < NC; ++ch) {
-          float v[16];
-          tc_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + ch * 16, v);
+          for (int c = 0; c < kBatch; ++c)
+            tc_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + (ch0 + c) * 16, v[c]);
           tc_wait_ld();
+          if (full) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = ch * 16 + i;
-            if (r < R && (full || j <= q_first + r % nrows)) tsc = fmaxf(tsc, v[i]);
+            for (int c = 0; c < kBatch; ++c)
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if ((ch0 + c) * 16 + i < R) tsc = fmaxf(tsc, v[c][i]);
+          } else {
+            for (int c = 0; c < kBatch; ++c)
+              for (int i = 0; i < 16; ++i)
+                if (rpos[(ch0 + c) * 16 + i] >= jrel) tsc = fmaxf(tsc, v[c][i]);
           }
         }
         float eps = kvalid ? eps_scale * __uint_as_float(kmag << 16) : 0.0f;
@@ -489,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         }
         const float dot = group_reduce_rows<8>(part, lane8);
         const int r = rc * 8 + lane8;
-        const bool ok = jok && r < R && j <= q_first + r % nrows;
+        const bool ok = jok && r < R && rpos[r] >= j - q_first;
         float v = ok ? dot : -INFINITY;
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
