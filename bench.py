@@ -204,7 +204,13 @@ class ClockSampler:
 # ---------------------------------------------------------------- distributed
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """Join the job's process group (one process per GPU; a no-op at N=1).
+
+    ``backend`` defaults to NCCL; gloo serves the CPU tests of these helpers.
+    The group's timeout is short so that ranks waiting on a lost peer end with
+    an error instead of hanging.
+    """
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -213,9 +219,12 @@ def dist_setup(n_gpus: int):
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -226,13 +235,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_us_per_layer(max_total_ms: float, steps: int, world: int) -> float:
+    """Whole-job decode throughput: every rank serves one layer per step, so
+    the job serves steps * world layers in the slowest rank's time."""
+    return max_total_ms * 1e3 / (steps * world)
 
 
 # ---------------------------------------------------------------- reference arm
@@ -280,7 +297,6 @@ def reference_arm(args, w: W.Workload, world: int, rank: int):
             idx, _, _, scored = oracle.mask(x["q"][0], x["k"], sh, units=pick, with_scored=True)
             full = np.full((units, idx.shape[1]), -1, np.int32)
             full[pick] = idx
-            sub = full[np.sort(pick)]
             flops = mask_algorithmic_flops(w, int(scored.sum()))
             for uu in np.sort(pick):
                 qb = uu % nqb
@@ -290,7 +306,6 @@ def reference_arm(args, w: W.Workload, world: int, rank: int):
                                 .reshape(-1)))
                 pos = np.arange(qb * w.block_q, min(qb * w.block_q + w.block_q, w.q_len))
                 flops += 4 * w.head_dim * w.group * int(np.searchsorted(keys, pos, side="right").sum())
-            del sub
         value, unit, hib = flops / (elapsed / args.steps) / 1e12, "TFLOP/s", True
     line = {"metric": METRIC, "value": value, "unit": unit, "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -472,7 +487,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     mask_ms = np.mean([ev[3 * l].elapsed_time(ev[3 * l + 1]) for l in range(layers)])
     attn_ms = np.mean([ev[3 * l + 1].elapsed_time(ev[3 * l + 2]) for l in range(layers)])
     total_ms = max_over_ranks(total_ms, world)
-    us_layer = total_ms * 1e3 / (steps * world)
+    us_layer = whole_job_us_per_layer(total_ms, steps, world)
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
     tensor_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
@@ -527,7 +542,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         barrier(world)
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), world)
         h2d = (q0.numel() + krow.numel() + vrow.numel()) * esz
-        e2e = {"value": e2e_ms * 1e3 / (steps * world), "unit": "us/layer",
+        e2e = {"value": whole_job_us_per_layer(e2e_ms, steps, world), "unit": "us/layer",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(q0.numel() * esz),
                "how": "CUDA graph of H2D (pinned) + hip_mask + hip_sparse_attn + D2H per step"}
         sess.check()
@@ -616,12 +631,14 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
 def main():
     args = parse()
     w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores alone; no process group
+        reference_arm(args, w, int(os.environ.get("WORLD_SIZE", "1")),
+                      int(os.environ.get("RANK", "0")))
+        return
     world, rank, local = dist_setup(args.gpus)
     try:
-        if args.impl == "reference":
-            reference_arm(args, w, world, rank)
-        else:
-            ours(args, w, world, rank, local)
+        ours(args, w, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
