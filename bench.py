@@ -376,17 +376,22 @@ def cpu_baseline(w: W.Workload, x: dict, min_seconds: float = 10.0):
 
 def traffic_from_profile(kernel: str, workload: str):
     """DRAM bytes per launch of ``kernel`` from the committed ncu summary, if
-    it was taken on the current source of the kernel; else None."""
+    it was taken on the current sources of the kernel; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f)
-    ent = d.get(f"{kernel}:{workload}")
+        ent = json.load(f).get("entries", {}).get(f"{kernel}:{workload}")
     if not ent:
         return None
-    src = os.path.join(ROOT, ent["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != ent["sha256"]:
+    h = hashlib.sha256()
+    for src in ent["sources"]:
+        p = os.path.join(ROOT, src)
+        if not os.path.exists(p):
+            return None
+        with open(p, "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != ent["sha256"]:
         return None
     return ent["dram_bytes_per_launch"]
 
