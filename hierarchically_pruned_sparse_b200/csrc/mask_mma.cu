@@ -9,26 +9,34 @@
 // CUDA-core kernel (mask_fma.cu).
 //
 // Design (one launch for all rounds; one cluster of C CTAs per mask row):
-//  * the representative key blocks of a round are gathered by cp.async into a
-//    ring of 128-key tiles laid out for the tensor core (K-major, 128-byte
-//    swizzle); the group's query rows (G heads x b_q positions, padded to N)
-//    sit in shared memory in the same layout for the whole launch;
-//  * one thread issues tcgen05.mma (M = 128 keys, N rows, K = 128, bf16 in,
-//    fp32 accumulate in TMEM); four warps read the 128 x N tile back
-//    (tcgen05.ld, one key per thread) and take the max over the valid rows;
-//  * each score t comes with a bound eps >= |t - s| on the distance to the
-//    canonical fp32 score s (the one the oracle ranks by): eps = gamma *
-//    max|k| * max_r sum|q_r| with gamma = 1024 * 2^-24, which covers an fp32
+//  * warps 5-7 gather the representative key blocks of a round by cp.async
+//    into a ring of 128-key tiles laid out for the tensor core (K-major,
+//    128-byte swizzle); the group's query rows (G heads x b_q positions,
+//    padded to N) sit in shared memory in the same layout for the whole
+//    launch;
+//  * one thread of warp 4 issues tcgen05.mma (M = 128 keys, N rows, K = 128,
+//    bf16 in, fp32 accumulate) into one of two TMEM accumulators, so the MMA
+//    of a tile overlaps the read-back of the one before; warps 0-3 read the
+//    128 x N tile back (tcgen05.ld, one key per thread) and take the max over
+//    the rows that see the key;
+//  * each score t comes with a bound eps >= |t - s| on its distance to the
+//    canonical fp32 score s (the one the oracle ranks by): per row,
+//    |t_r - s_r| <= gamma * sum_i |q_ri k_i| <= gamma * |q_r|_2 |k|_2
+//    (Cauchy-Schwarz) with gamma = 1024 * 2^-24, which covers an fp32
 //    accumulation of the 128 exact bf16 products in any order (<= 2^-23 per
-//    addition) plus the canonical order's own rounding;
+//    addition) plus the canonical order's own rounding; the max over rows
+//    moves by at most the largest row bound;
 //  * selection: theta = the n0-th largest t (bucket select, as in
 //    mask_fma.cu) and eps_max = max eps. A candidate with t - eps > theta +
 //    eps_max is above the canonical cut for sure, one with t + eps < theta -
 //    eps_max below it for sure; only the few in between (the band) are
-//    re-scored in the canonical fp32 order on CUDA cores (keys re-read from
-//    global memory, where they are hot in L2), and the band's best take the
-//    remaining places by (score desc, start asc). The result equals the
-//    selection by canonical scores exactly.
+//    re-scored in the canonical fp32 order on CUDA cores, and the band's best
+//    take the remaining places by (score desc, start asc). The result equals
+//    the selection by canonical scores exactly;
+//  * re-scoring the band: with few rows (N <= 32) every row of every band key
+//    is re-scored. With many rows the band's keys get one more MMA, and only
+//    the rows that can hold the maximum are re-scored: row r of the candidate
+//    with t_r + eps_r < max_r' (t_r' - eps_r') has s_r < s.
 #include <cooperative_groups.h>
 
 #include "hips_common.cuh"
@@ -46,12 +54,22 @@ constexpr int kTileBytes = kM * 256;    // bf16 key rows
 constexpr int kHalfBytes = kTileBytes / 2;
 constexpr int kBuckets = 2048;
 constexpr float kGamma = 1024.0f / 16777216.0f;
+// an fp32 sum of 128 squares and its square root are within 2^-16 of the
+// true norm; the factor makes the computed norms upper bounds
+constexpr float kNormUp = 1.0f + 1.0f / 4096.0f;
+constexpr int kIssuerWarp = 4;          // lane 0 issues the MMAs
+constexpr int kProducerWarp0 = 5;       // warps 5-7 gather key tiles
+constexpr int kProducers = (kWarps - kProducerWarp0) * 32;
 
-__host__ __device__ constexpr int stages_for(int nc) { return nc >= 16 ? 2 : nc >= 8 ? 3 : 4; }
-__host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 16 < 32 ? 32 : nc * 16; }
+__host__ __device__ constexpr int stages_for(int nc, int per) {
+  return per > 8 ? 2 : nc >= 16 ? 2 : nc >= 8 ? 3 : 4;
+}
+__host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 32 < 32 ? 32 : nc * 32; }
+__host__ __device__ constexpr int mask_words(int nc) { return nc < 2 ? 1 : nc / 2; }
 
 struct MmaSmem {
-  int ring, bq, bar, slot, rpos, cs, ce, keepb, band, band_key, xch, hist, scratch, total;
+  int ring, bq, bar, slot, rpos, qn, cs, ce, keepb, band, band_key, xch, hist, rowmask, scratch,
+      total;
 };
 
 __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
@@ -60,23 +78,25 @@ __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
 // copy and writes the next round's list into the other. xch holds the (score,
 // bound) of every candidate of a round: each CTA writes its own candidates
 // into every CTA of the cluster; two copies alternate between rounds.
-__host__ __device__ inline MmaSmem mma_layout(int nc, int n0max, int per_cta, int cluster) {
+__host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cluster) {
   MmaSmem L;
   const int n = 2 * n0max;
+  const int S = stages_for(nc, per);
   int o = 0;
-  L.ring = o;     o += stages_for(nc) * kTileBytes;
+  L.ring = o;     o += S * kTileBytes;
   L.bq = o;       o += nc * 16 * 256;
-  L.bar = o;      o += 16;
+  L.bar = o;      o += 8 * (2 * S + 5);
   L.slot = o;     o += 16;
   L.rpos = o;     o += nc * 16 * 4;  // query position offset (r % b_q) of operand row r
+  L.qn = o;       o += nc * 16 * 4;  // |q_r|_2, rounded up (0 for padding rows)
   L.cs = o;       o += 2 * al(n * 4, 16);
   L.ce = o;       o += 2 * al(n * 4, 16);
   L.keepb = o;    o += al(n, 16);
   L.band = o;     o += al(n * 4, 16);
   L.band_key = o; o += al(n * 4, 16);
   L.xch = o;      o += (cluster > 1 ? 2 : 1) * al(n * 8, 16);
-  (void)per_cta;
   L.hist = o;     o += kBuckets * 4;
+  L.rowmask = o;  o += nc >= 4 ? kM * mask_words(nc) * 4 : 0;
   L.scratch = o;  o += 64 * 4;
   L.total = o + 1024;  // room to align the base to 1024 bytes
   return L;
@@ -111,11 +131,64 @@ __device__ int find_cut(const int* hist, int n, int* scratch) {
   return scratch[40];
 }
 
+// The 16 elements lane8 owns in the canonical order (slices lane8 and
+// lane8 + 8 of 8 elements) of row r of a swizzled K-major operand whose two
+// 64-element halves are rows * 128 bytes apart.
+__device__ __forceinline__ void load_row16_sw(const unsigned char* base, int rows, int r, int lane8,
+                                              float (&x)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(base + sw128_offset(r, lane8));
+  const uint4 b = *reinterpret_cast<const uint4*>(base + rows * 128 + sw128_offset(r, lane8));
+  x[0] = bf16lo(a.x); x[1] = bf16hi(a.x); x[2] = bf16lo(a.y); x[3] = bf16hi(a.y);
+  x[4] = bf16lo(a.z); x[5] = bf16hi(a.z); x[6] = bf16lo(a.w); x[7] = bf16hi(a.w);
+  x[8] = bf16lo(b.x); x[9] = bf16hi(b.x); x[10] = bf16lo(b.y); x[11] = bf16hi(b.y);
+  x[12] = bf16lo(b.z); x[13] = bf16hi(b.z); x[14] = bf16lo(b.w); x[15] = bf16hi(b.w);
+}
+
+// Squared 2-norm of key row kk of a swizzled tile.
+__device__ __forceinline__ float tile_row_norm2(const unsigned char* tile, int kk) {
+  float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) {
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + (ch >> 3) * kHalfBytes +
+                                                    sw128_offset(kk, ch & 7));
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = bf16lo(x[q]), hi = bf16hi(x[q]);
+      s0 = fmaf(lo, lo, s0);
+      s1 = fmaf(hi, hi, s1);
+    }
+  }
+  return s0 + s1;
+}
+
+// Gather `nkeys` key rows into a swizzled tile: key kk is row key_of(kk) of
+// the head (skipped when >= Tc). Thread p of `nthr` copies half of the 16-byte
+// chunks of key p / 2 (+ nthr / 2, ...): two neighbouring threads read one
+// 32-byte sector.
+template <typename KeyOf>
+__device__ __forceinline__ void gather_tile(unsigned char* tile, const unsigned char* kbase,
+                                            int nkeys, int p, int nthr, int64_t Tc,
+                                            KeyOf key_of) {
+  for (int kk = p >> 1; kk < nkeys; kk += nthr >> 1) {
+    const int64_t j = key_of(kk);
+    if (j < Tc) {
+      const unsigned char* src = kbase + j * 256;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int ch = (p & 1) + 2 * i;
+        cp_async16(tile + (ch >> 3) * kHalfBytes + sw128_offset(kk, ch & 7), src + ch * 16);
+      }
+    }
+  }
+}
+
 template <int NC, int PER>
 __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   constexpr int N = NC * 16;
-  constexpr int S = stages_for(NC);
+  constexpr int S = stages_for(NC, PER);
   constexpr int TCOLS = tmem_cols_for(NC);
+  constexpr int MW = mask_words(NC);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int C = a.cluster;
@@ -139,13 +212,18 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   const int per_cta = a.per_cta;
   const int nbuf = 2 * a.n0max;  // stride between the two candidate buffers
 
-  const MmaSmem L = mma_layout(NC, a.n0max, per_cta, C);
+  const MmaSmem L = mma_layout(NC, PER, a.n0max, C);
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   unsigned char* ring = smem + L.ring;
   unsigned char* bq = smem + L.bq;
-  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);  // [S]: tile landed
+  uint64_t* empty = full + S;        // [S]: tile read (MMA and norms done)
+  uint64_t* mma_done = empty + S;    // [2]: accumulator written
+  uint64_t* tm_empty = mma_done + 2; // [2]: accumulator read back
+  uint64_t* band_bar = tm_empty + 2; // band MMA done
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.slot);
   int* rpos = reinterpret_cast<int*>(smem + L.rpos);
+  float* qn = reinterpret_cast<float*>(smem + L.qn);
   int* cs_all = reinterpret_cast<int*>(smem + L.cs);
   int* ce_all = reinterpret_cast<int*>(smem + L.ce);
   uint8_t* keepb = reinterpret_cast<uint8_t*>(smem + L.keepb);
@@ -153,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   uint32_t* band_key = reinterpret_cast<uint32_t*>(smem + L.band_key);
   float2* xch = reinterpret_cast<float2*>(smem + L.xch);
   int* hist = reinterpret_cast<int*>(smem + L.hist);
+  uint32_t* rowmask = reinterpret_cast<uint32_t*>(smem + L.rowmask);
   int* scratch = reinterpret_cast<int*>(smem + L.scratch);
   float* fscratch = reinterpret_cast<float*>(scratch);
   uint32_t* uscratch = reinterpret_cast<uint32_t*>(scratch);
@@ -162,7 +241,15 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
                                (static_cast<int64_t>(b) * a.n_kvheads + g) * a.kv_cap * 256;
 
   if (tid == 0) {
-    mbar_init(mma_bar, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], kProducers);
+      mbar_init(&empty[s], 4);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&mma_done[s], 1);
+      mbar_init(&tm_empty[s], 4);
+    }
+    mbar_init(band_bar, 1);
     fence_mbar_init();
   }
   __syncwarp();
@@ -181,6 +268,20 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   }
   for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
   for (int r = tid; r < N; r += kThreads) rpos[r] = r < R ? r % nrows : -1;  // -1: padding row
+  // |q_r|_2 of every row (one warp per row), rounded up
+  for (int r = warp; r < N; r += kWarps) {
+    float s = 0.0f;
+    if (r < R) {
+      const int h = g * a.group + r / nrows, qi = i0 + r % nrows;
+      const uint2 w = *reinterpret_cast<const uint2*>(
+          qg + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + qi) * kD + lane * 4);
+      const float x0 = bf16lo(w.x), x1 = bf16hi(w.x), x2 = bf16lo(w.y), x3 = bf16hi(w.y);
+      s = fmaf(x0, x0, fmaf(x1, x1, fmaf(x2, x2, x3 * x3)));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) qn[r] = r < R ? sqrtf(s) * kNormUp : 0.0f;
+  }
 
   // ---- candidates of round 1: the halves of the n0 initial chunks
   // (a one-block chunk stays whole); thread t owns chunks [t*pc, (t+1)*pc)
@@ -215,32 +316,20 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       }
     }
   }
-  // max over the rows of sum_i |q_ri| (rounded up)
-  float q1 = 0.0f;
-  for (int r = tid; r < R; r += kThreads) {
-    const int h = g * a.group + r / nrows, qi = i0 + r % nrows;
-    const uint16_t* row = qg + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + qi) * kD;
-    float s = 0.0f;
-    for (int e = 0; e < kD; ++e) s += fabsf(__uint_as_float(static_cast<uint32_t>(row[e]) << 16));
-    q1 = fmaxf(q1, s * (1.0f + 512.0f / 16777216.0f));
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) q1 = fmaxf(q1, __shfl_xor_sync(0xffffffffu, q1, o));
-  if (lane == 0) fscratch[48 + warp] = q1;
   fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tslot;
-  float q1max = fscratch[48];
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) q1max = fmaxf(q1max, fscratch[48 + w]);
-  const float eps_scale = kGamma * q1max;
+  float q2max = 0.0f;
+  for (int r = 0; r < N; ++r) q2max = fmaxf(q2max, qn[r]);
+  const float eps_scale = kGamma * q2max;  // times |k|_2 (rounded up)
   const uint32_t idesc = idesc_bf16_f32(kM, N);
   const int cpt = kM >> lbk;  // candidates per tile
-  uint32_t mma_phase = 0;
+  int gt = 0;                 // tiles of earlier rounds (pipeline position)
+  uint32_t band_phase = 0;
   int cur = 0, buf = 0;
-  bool timed_out = false;
+  bool timed_out = false;  // once a wait gave up, this thread waits no more
 
   while (nlong > 0) {
     const int* cs = cs_all + cur * nbuf;
@@ -255,47 +344,44 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     const int ntiles = (c_hi - c_lo + cpt - 1) / cpt;
     float2* my_x = xch + buf * nbuf;  // indexed by candidate
 
-    // all threads: gather tile t (if any) into its ring slot, commit a group;
-    // thread t copies chunk (t % 16) of keys t/16, t/16 + 16, ... of the tile
-    auto issue = [&](int t) {
-      if (t < ntiles) {
-        unsigned char* dst = ring + (t % S) * kTileBytes;
+    if (warp >= kProducerWarp0) {
+      // ---------------- gather tiles into the ring
+      const int p = tid - kProducerWarp0 * 32;
+      for (int t = 0; t < ntiles; ++t) {
+        const int gi = gt + t, slot = gi % S;
+        if (gi >= S && !timed_out && !mbar_wait(&empty[slot], ((gi / S) - 1) & 1)) timed_out = true;
         const int cf = c_lo + t * cpt;
         const int nkeys = min(cpt, c_hi - cf) << lbk;
-        const int ch = tid & 15;
-        unsigned char* dch = dst + (ch >> 3) * kHalfBytes;
+        gather_tile(ring + slot * kTileBytes, kbase, nkeys, p, kProducers, Tc,
+                    [&](int kk) { return rep_key(cf + (kk >> lbk)) + (kk & (bk - 1)); });
+        cp_async_arrive(&full[slot]);
+      }
+    } else if (warp == kIssuerWarp) {
+      // ---------------- MMA issue (one thread)
+      if (lane == 0) {
+        for (int t = 0; t < ntiles; ++t) {
+          const int gi = gt + t, slot = gi % S, tb = gi & 1;
+          if (!timed_out && !mbar_wait(&full[slot], (gi / S) & 1)) timed_out = true;
+          if (gi >= 2 && !timed_out && !mbar_wait(&tm_empty[tb], ((gi >> 1) - 1) & 1)) timed_out = true;
+          tc_fence_after_sync();
+          fence_proxy_async_smem();  // the gathered rows -> tensor-core reads
+          const unsigned char* tile = ring + slot * kTileBytes;
 #pragma unroll
-        for (int m = 0; m < kM / 16; ++m) {
-          const int kk = (tid >> 4) + 16 * m;
-          if (kk < nkeys) {
-            const int64_t j = rep_key(cf + (kk >> lbk)) + (kk & (bk - 1));
-            if (j < Tc) cp_async16(dch + sw128_offset(kk, ch & 7), kbase + j * 256 + ch * 16);
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t a_addr = smem_u32(tile + (k >> 2) * kHalfBytes) + (k & 3) * 32;
+            const uint32_t b_addr = smem_u32(bq + (k >> 2) * (N * 128)) + (k & 3) * 32;
+            tc_mma_bf16(tmem + tb * N, sw128_desc(a_addr), sw128_desc(b_addr), idesc, k > 0);
           }
+          tc_commit(&mma_done[tb]);
         }
       }
-      cp_async_commit();
-    };
-
-    for (int t = 0; t < S; ++t) issue(t);
-    for (int t = 0; t < ntiles; ++t) {
-      cp_async_wait<S - 1>();
-      fence_proxy_async_smem();
-      tc_fence_before_sync();
-      __syncthreads();
-      const unsigned char* tile = ring + (t % S) * kTileBytes;
-      if (tid == 0) {
-        tc_fence_after_sync();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t a_addr = smem_u32(tile + (k >> 2) * kHalfBytes) + (k & 3) * 32;
-          const uint32_t b_addr = smem_u32(bq + (k >> 2) * (N * 128)) + (k & 3) * 32;
-          tc_mma_bf16(tmem, sw128_desc(a_addr), sw128_desc(b_addr), idesc, k > 0);
-        }
-        tc_commit(mma_bar);
-      }
-      if (warp < 4) {
+      __syncwarp();
+    } else {
+      // ---------------- read back: thread = key kk of the tile
+      const int kk = warp * 32 + lane;
+      for (int t = 0; t < ntiles; ++t) {
+        const int gi = gt + t, slot = gi % S, tb = gi & 1;
         const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
-        const int kk = warp * 32 + lane;
         const int lc = kk >> lbk;
         bool kvalid = lc < cc;
         int64_t j = 0;
@@ -303,34 +389,24 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
           j = rep_key(cf + lc) + (kk & (bk - 1));
           kvalid = j < Tc;
         }
-        // max |k| of this key row (bf16 magnitudes compare as integers)
-        uint32_t kmag = 0;
-        if (kvalid) {
-#pragma unroll
-          for (int ch = 0; ch < 16; ++ch) {
-            const uint4 w = *reinterpret_cast<const uint4*>(tile + (ch >> 3) * kHalfBytes +
-                                                            sw128_offset(kk, ch & 7));
-            const uint32_t x[4] = {w.x & 0x7fff7fffu, w.y & 0x7fff7fffu, w.z & 0x7fff7fffu,
-                                   w.w & 0x7fff7fffu};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) kmag = max(kmag, max(x[q] & 0xffffu, x[q] >> 16));
-          }
-        }
-        if (!mbar_wait(mma_bar, mma_phase)) timed_out = true;
+        if (!timed_out && !mbar_wait(&full[slot], (gi / S) & 1)) timed_out = true;
+        // |k|_2 while the MMA runs
+        const float kn2 = kvalid ? tile_row_norm2(ring + slot * kTileBytes, kk) : 0.0f;
+        if (!timed_out && !mbar_wait(&mma_done[tb], (gi >> 1) & 1)) timed_out = true;
         tc_fence_after_sync();
         __syncwarp();
         float tsc = -INFINITY;
-        const bool full = j <= q_first;  // every row sees this key
-        const int64_t jrel = j - q_first;   // otherwise row r needs r % b_q >= jrel
+        const bool all_rows = j <= q_first;  // every row sees this key
+        const int64_t jrel = j - q_first;    // otherwise row r needs r % b_q >= jrel
         constexpr int kBatch = NC < 4 ? NC : 4;
 #pragma unroll 1
         for (int ch0 = 0; ch0 < NC; ch0 += kBatch) {
           float v[kBatch][16];
 #pragma unroll
           for (int c = 0; c < kBatch; ++c)
-            tc_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + (ch0 + c) * 16, v[c]);
+            tc_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + tb * N + (ch0 + c) * 16, v[c]);
           tc_wait_ld();
-          if (full) {
+          if (all_rows) {
 #pragma unroll
             for (int c = 0; c < kBatch; ++c)
 #pragma unroll
@@ -342,7 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
                 if (rpos[(ch0 + c) * 16 + i] >= jrel) tsc = fmaxf(tsc, v[c][i]);
           }
         }
-        float eps = kvalid ? eps_scale * __uint_as_float(kmag << 16) : 0.0f;
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&empty[slot]);
+          mbar_arrive(&tm_empty[tb]);
+        }
+        float eps = kvalid ? eps_scale * (sqrtf(kn2) * kNormUp) : 0.0f;
         if (!kvalid) tsc = -INFINITY;
         for (int o = 1; o < bk; o <<= 1) {
           tsc = fmaxf(tsc, __shfl_xor_sync(0xffffffffu, tsc, o));
@@ -355,15 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
             if (p != rank) *cluster.map_shared_rank(my_x + cf + lc, p) = val;
         }
       }
-      mma_phase ^= 1u;
-      tc_fence_before_sync();
-      __syncthreads();
-      issue(t + S);  // into the slot just consumed
     }
+    gt += ntiles;
 
     if (tid == 0 && a.status && c_hi > c_lo)
       atomicAdd(&a.status->scored, static_cast<unsigned long long>(c_hi - c_lo));
     // ---- all scores are local now; thread t owns candidates [t*PER, (t+1)*PER)
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
     if (C > 1) cluster.sync();
     float tv[PER], ev[PER];
     const int ibase = tid * PER;
@@ -469,8 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     for (int m = tid; m < nband; m += kThreads) band_key[m] = 0u;
     __syncthreads();
 
-    // ---- canonical fp32 scores of the band (8 lanes per key, 8 rows per group)
-    {
+    if constexpr (NC < 4) {
+      // ---- canonical fp32 scores of the band: every row of every key
+      // (8 lanes per key, 8 rows per group; keys read from global memory)
       const int nrc = (R + 7) / 8;
       const int items = nband * bk * nrc;
       for (int base = warp * 4; base < items; base += kWarps * 4) {  // warp-uniform loop
@@ -489,12 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         for (int rr = 0; rr < 8; ++rr) {
           const int r = min(rc * 8 + rr, N - 1);
           float qv[16];
-          const uint4 x0 = *reinterpret_cast<const uint4*>(bq + sw128_offset(r, lane8));
-          const uint4 x1 = *reinterpret_cast<const uint4*>(bq + N * 128 + sw128_offset(r, lane8));
-          qv[0] = bf16lo(x0.x); qv[1] = bf16hi(x0.x); qv[2] = bf16lo(x0.y); qv[3] = bf16hi(x0.y);
-          qv[4] = bf16lo(x0.z); qv[5] = bf16hi(x0.z); qv[6] = bf16lo(x0.w); qv[7] = bf16hi(x0.w);
-          qv[8] = bf16lo(x1.x); qv[9] = bf16hi(x1.x); qv[10] = bf16lo(x1.y); qv[11] = bf16hi(x1.y);
-          qv[12] = bf16lo(x1.z); qv[13] = bf16hi(x1.z); qv[14] = bf16lo(x1.w); qv[15] = bf16hi(x1.w);
+          load_row16_sw(bq, N, r, lane8, qv);
           float acc = 0.0f;
 #pragma unroll
           for (int e = 0; e < 16; ++e) acc = __fmaf_rn(qv[e], kx[e], acc);
@@ -508,6 +586,117 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
         if (lane8 == 0 && live && v > -INFINITY) atomicMax(&band_key[m], score_key(v));
+      }
+    } else {
+      // ---- canonical fp32 scores of the band, rows that can hold the max only
+      const int bpt = kM >> lbk;  // band members per tile
+      unsigned char* tile = ring;   // every ring slot is free between rounds
+      for (int m0 = 0; m0 < nband; m0 += bpt) {
+        const int mcnt = min(bpt, nband - m0);
+        const int nkeys = mcnt << lbk;
+        gather_tile(tile, kbase, nkeys, tid, kThreads, Tc,
+                    [&](int kk) { return rep_key(band[m0 + (kk >> lbk)]) + (kk & (bk - 1)); });
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+          tc_fence_after_sync();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t a_addr = smem_u32(tile + (k >> 2) * kHalfBytes) + (k & 3) * 32;
+            const uint32_t b_addr = smem_u32(bq + (k >> 2) * (N * 128)) + (k & 3) * 32;
+            tc_mma_bf16(tmem, sw128_desc(a_addr), sw128_desc(b_addr), idesc, k > 0);
+          }
+          tc_commit(band_bar);
+        }
+        if (warp < 4) {
+          const int kk = warp * 32 + lane;
+          const int lm = kk >> lbk;
+          bool kvalid = lm < mcnt;
+          int64_t j = 0;
+          if (kvalid) {
+            j = rep_key(band[m0 + lm]) + (kk & (bk - 1));
+            kvalid = j < Tc;
+          }
+          const float kb = kvalid ? kGamma * sqrtf(tile_row_norm2(tile, kk)) * kNormUp : 0.0f;
+          if (!timed_out && !mbar_wait(band_bar, band_phase)) timed_out = true;
+          tc_fence_after_sync();
+          __syncwarp();
+          const int64_t jrel = kvalid ? j - q_first : (int64_t{1} << 40);
+          const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+          // pass 1: the largest lower bound t_r - eps_r over the rows seeing the key
+          float tstar = -INFINITY;
+#pragma unroll 1
+          for (int ch = 0; ch < NC; ++ch) {
+            float v[16];
+            tc_ld16(taddr + ch * 16, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int r = ch * 16 + i;
+              if (r < R && rpos[r] >= jrel) tstar = fmaxf(tstar, v[i] - kb * qn[r]);
+            }
+          }
+          for (int o = 1; o < bk; o <<= 1) tstar = fmaxf(tstar, __shfl_xor_sync(0xffffffffu, tstar, o));
+          // pass 2: the rows whose upper bound t_r + eps_r reaches it
+          uint32_t mw[MW];
+#pragma unroll
+          for (int w = 0; w < MW; ++w) mw[w] = 0u;
+#pragma unroll
+          for (int ch = 0; ch < NC; ++ch) {
+            float v[16];
+            tc_ld16(taddr + ch * 16, v);
+            tc_wait_ld();
+            uint32_t bits = 0u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int r = ch * 16 + i;
+              if (r < R && rpos[r] >= jrel && v[i] + kb * qn[r] >= tstar) bits |= 1u << i;
+            }
+            mw[ch >> 1] |= bits << ((ch & 1) * 16);
+          }
+#pragma unroll
+          for (int w = 0; w < MW; ++w) rowmask[kk * MW + w] = mw[w];
+          tc_fence_before_sync();
+        }
+        __syncthreads();
+        // one warp per key; each 8-lane group re-scores one marked row at a time
+        for (int kk = warp; kk < nkeys; kk += kWarps) {
+          float kx[16];
+          load_row16_sw(tile, kHalfBytes / 128, kk, lane8, kx);
+          float best = -INFINITY;
+          for (int w = 0; w < MW; ++w) {
+            uint32_t bits = rowmask[kk * MW + w];  // the same in every lane
+            while (bits) {
+              int r = -1;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (bits) {
+                  if (q == grp) r = w * 32 + __ffs(bits) - 1;
+                  bits &= bits - 1;
+                }
+              }
+              float acc = 0.0f;
+              if (r >= 0) {
+                float qv[16];
+                load_row16_sw(bq, N, r, lane8, qv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc = __fmaf_rn(qv[e], kx[e], acc);
+              }
+              acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+              acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+              acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+              if (r >= 0) best = fmaxf(best, acc);
+            }
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+          if (lane == 0 && best > -INFINITY) atomicMax(&band_key[m0 + (kk >> lbk)], score_key(best));
+        }
+        band_phase ^= 1u;
+        __syncthreads();
       }
     }
     __syncthreads();
@@ -680,7 +869,8 @@ int mask_mma_nc(int rows_max) {
 }
 
 int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster) {
-  return mma_layout(nc, n0max, per_cta, cluster).total;
+  (void)per_cta;
+  return mma_layout(nc, n0max <= 1024 ? 8 : 16, n0max, cluster).total;
 }
 
 int mask_mma_tile_keys() { return kM; }
