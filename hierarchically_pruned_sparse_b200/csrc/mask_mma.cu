@@ -146,7 +146,9 @@ __device__ __forceinline__ void load_row16_sw(const unsigned char* base, int row
 
 // Squared 2-norm of key row kk of a swizzled tile.
 __device__ __forceinline__ float tile_row_norm2(const unsigned char* tile, int kk) {
-  float s0 = 0.0f, s1 = 0.0f;
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
 #pragma unroll
   for (int ch = 0; ch < 16; ++ch) {
     const uint4 w = *reinterpret_cast<const uint4*>(tile + (ch >> 3) * kHalfBytes +
@@ -155,12 +157,59 @@ __device__ __forceinline__ float tile_row_norm2(const unsigned char* tile, int k
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float lo = bf16lo(x[q]), hi = bf16hi(x[q]);
-      s0 = fmaf(lo, lo, s0);
-      s1 = fmaf(hi, hi, s1);
+      acc[2 * q] = fmaf(lo, lo, acc[2 * q]);
+      acc[2 * q + 1] = fmaf(hi, hi, acc[2 * q + 1]);
     }
   }
-  return s0 + s1;
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
+
+// Max of 16 values as a tree (depth 4).
+__device__ __forceinline__ float max16(const float (&v)[16]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(v[i], v[i + 8]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
+  return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
+}
+
+// Largest accumulator column of this thread's TMEM lane over the operand rows
+// that see key j: rows [0, R) when every row does (all_rows), else the rows r
+// with rpos[r] >= jrel. Warp-collective (every lane of the warp calls it).
+template <int NC>
+__device__ __forceinline__ float tmem_row_max(uint32_t taddr, int R, bool all_rows, int64_t jrel,
+                                              const int* rpos) {
+  constexpr int kBatch = NC < 4 ? NC : 4;
+  float acc[kBatch];
+#pragma unroll
+  for (int c = 0; c < kBatch; ++c) acc[c] = -INFINITY;
+#pragma unroll 1
+  for (int ch0 = 0; ch0 < NC; ch0 += kBatch) {
+    float v[kBatch][16];
+#pragma unroll
+    for (int c = 0; c < kBatch; ++c) tc_ld16(taddr + (ch0 + c) * 16, v[c]);
+    tc_wait_ld();
+#pragma unroll
+    for (int c = 0; c < kBatch; ++c) {
+      const int r0 = (ch0 + c) * 16;
+      if (all_rows && r0 + 16 <= R) {
+        acc[c] = fmaxf(acc[c], max16(v[c]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const bool ok = r0 + i < R && (all_rows || rpos[r0 + i] >= jrel);
+          if (ok) acc[c] = fmaxf(acc[c], v[c][i]);
+        }
+      }
+    }
+  }
+  float m = acc[0];
+#pragma unroll
+  for (int c = 1; c < kBatch; ++c) m = fmaxf(m, acc[c]);
+  return m;
+}
+
 
 // Gather `nkeys` key rows into a swizzled tile: key kk is row key_of(kk) of
 // the head (skipped when >= Tc). Thread p of `nthr` copies half of the 16-byte
@@ -395,27 +444,29 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         if (!timed_out && !mbar_wait(&mma_done[tb], (gi >> 1) & 1)) timed_out = true;
         tc_fence_after_sync();
         __syncwarp();
+        // every row sees key j when j <= q_first; else row r needs r % b_q >= j - q_first
         float tsc = -INFINITY;
-        const bool all_rows = j <= q_first;  // every row sees this key
-        const int64_t jrel = j - q_first;    // otherwise row r needs r % b_q >= jrel
-        constexpr int kBatch = NC < 4 ? NC : 4;
-#pragma unroll 1
-        for (int ch0 = 0; ch0 < NC; ch0 += kBatch) {
-          float v[kBatch][16];
+        if constexpr (NC >= 4) {
+          tsc = tmem_row_max<NC>(tmem + (static_cast<uint32_t>(warp * 32) << 16) + tb * N, R,
+                                 j <= q_first, j - q_first, rpos);
+        } else {
+          const bool all_rows = j <= q_first;
+          const int64_t jrel = j - q_first;
+          float v[NC][16];
 #pragma unroll
-          for (int c = 0; c < kBatch; ++c)
-            tc_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + tb * N + (ch0 + c) * 16, v[c]);
+          for (int c = 0; c < NC; ++c)
+            tc_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + tb * N + c * 16, v[c]);
           tc_wait_ld();
           if (all_rows) {
 #pragma unroll
-            for (int c = 0; c < kBatch; ++c)
+            for (int c = 0; c < NC; ++c)
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                if ((ch0 + c) * 16 + i < R) tsc = fmaxf(tsc, v[c][i]);
+                if (c * 16 + i < R) tsc = fmaxf(tsc, v[c][i]);
           } else {
-            for (int c = 0; c < kBatch; ++c)
+            for (int c = 0; c < NC; ++c)
               for (int i = 0; i < 16; ++i)
-                if (rpos[(ch0 + c) * 16 + i] >= jrel) tsc = fmaxf(tsc, v[c][i]);
+                if (rpos[c * 16 + i] >= jrel) tsc = fmaxf(tsc, v[c][i]);
           }
         }
         tc_fence_before_sync();
@@ -620,27 +671,19 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
             j = rep_key(band[m0 + lm]) + (kk & (bk - 1));
             kvalid = j < Tc;
           }
-          const float kb = kvalid ? kGamma * sqrtf(tile_row_norm2(tile, kk)) * kNormUp : 0.0f;
+          const float ek = kvalid ? eps_scale * (sqrtf(tile_row_norm2(tile, kk)) * kNormUp) : 0.0f;
           if (!timed_out && !mbar_wait(band_bar, band_phase)) timed_out = true;
           tc_fence_after_sync();
           __syncwarp();
-          const int64_t jrel = kvalid ? j - q_first : (int64_t{1} << 40);
+          const bool all_rows = j <= q_first;
+          const int64_t jrel = j - q_first;
           const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-          // pass 1: the largest lower bound t_r - eps_r over the rows seeing the key
-          float tstar = -INFINITY;
-#pragma unroll 1
-          for (int ch = 0; ch < NC; ++ch) {
-            float v[16];
-            tc_ld16(taddr + ch * 16, v);
-            tc_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int r = ch * 16 + i;
-              if (r < R && rpos[r] >= jrel) tstar = fmaxf(tstar, v[i] - kb * qn[r]);
-            }
-          }
+          // s >= max over the candidate's keys of (t_max - eps): rows below
+          // that by more than their key's eps cannot hold the maximum
+          const float tmax = tmem_row_max<NC>(taddr, R, all_rows, jrel, rpos);  // every lane
+          float tstar = kvalid ? tmax - ek : -INFINITY;
           for (int o = 1; o < bk; o <<= 1) tstar = fmaxf(tstar, __shfl_xor_sync(0xffffffffu, tstar, o));
-          // pass 2: the rows whose upper bound t_r + eps_r reaches it
+          const float thr = tstar - ek;
           uint32_t mw[MW];
 #pragma unroll
           for (int w = 0; w < MW; ++w) mw[w] = 0u;
@@ -653,7 +696,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int r = ch * 16 + i;
-              if (r < R && rpos[r] >= jrel && v[i] + kb * qn[r] >= tstar) bits |= 1u << i;
+              const bool ok = kvalid && r < R && (all_rows || rpos[r] >= jrel);
+              bits |= (ok && v[i] >= thr) ? (1u << i) : 0u;
             }
             mw[ch >> 1] |= bits << ((ch & 1) * 16);
           }
