@@ -3,8 +3,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--layers L]
 
-One step is one pass of the whole hot path (hip_mask + hip_sparse_attn, i.e.
-one attention layer) over one batch of the workload. The default workload is
+One step is one pass of the whole hot path (a fresh mask and the sparse
+attention over it, i.e. one attention layer) over one batch of the workload:
+hip_mask_sparse_attn for decode (one launch for bf16 groups of <= 4 query
+rows; --two-calls times hip_mask + hip_sparse_attn instead), hip_mask +
+hip_sparse_attn for prefill. The default workload is
 Llama-3.1-8B-shaped decode at T = 128k (32 query / 8 KV heads, d = 128,
 k = 2048, b_k = 2, sink 128 + window 1024, bf16). Inputs are synthetic
 (seeded AR(1) keys/values, Gaussian queries, needle keys) and resident in
@@ -55,6 +58,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="rotating layer buffers (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--two-calls", action="store_true",
+                    help="decode: time hip_mask + hip_sparse_attn instead of hip_mask_sparse_attn")
     return ap.parse_args()
 
 
@@ -425,9 +430,21 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     idxs = [sess.new_idx() for _ in range(layers)]
     outs = [torch.empty_like(q0) for _ in range(layers)]
 
-    def step(l):
+    # decode steps go through hip_mask_sparse_attn (a fresh mask and the
+    # attention over it); the library runs it as one launch for bf16 groups of
+    # at most 4 query rows, as the two kernels otherwise
+    fused = not prefill and not args.two_calls
+    one_launch = fused and w.dtype == "bf16" and w.group * min(w.block_q, w.q_len) <= 4
+
+    def two_calls(l):
         hb.hip_mask(qs[l], ks[l], sess.p, idxs[l])
         hb.hip_sparse_attn(qs[l], ks[l], vs[l], idxs[l], sess.p, outs[l])
+
+    def step(l):
+        if fused:
+            hb.hip_mask_sparse_attn(qs[l], ks[l], vs[l], sess.p, idxs[l], outs[l])
+        else:
+            two_calls(l)
 
     with torch.cuda.stream(stream):
         for i in range(max(args.warmup, 3)):
@@ -450,15 +467,23 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
 
     # CUDA graphs of `layers` steps (and of the remainder of K), with
     # per-kernel events in the full graph
+    def graph_with_events(ev, fused_step):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for l in range(layers):
+                ev[3 * l].record(stream)
+                if fused_step:
+                    hb.hip_mask_sparse_attn(qs[l], ks[l], vs[l], sess.p, idxs[l], outs[l])
+                    ev[3 * l + 1].record(stream)
+                else:
+                    hb.hip_mask(qs[l], ks[l], sess.p, idxs[l])
+                    ev[3 * l + 1].record(stream)
+                    hb.hip_sparse_attn(qs[l], ks[l], vs[l], idxs[l], sess.p, outs[l])
+                ev[3 * l + 2].record(stream)
+        return gr
+
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * layers)]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for l in range(layers):
-            ev[3 * l].record(stream)
-            hb.hip_mask(qs[l], ks[l], sess.p, idxs[l])
-            ev[3 * l + 1].record(stream)
-            hb.hip_sparse_attn(qs[l], ks[l], vs[l], idxs[l], sess.p, outs[l])
-            ev[3 * l + 2].record(stream)
+    g = graph_with_events(ev, fused)
     steps = max(1, args.steps)
     reps, rem = divmod(steps, layers)
     g_rem = None
@@ -502,7 +527,23 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     mask_tf = mask_flops / (mask_ms * 1e-3) / 1e12
     attn_tf = attn_flops / (attn_ms * 1e-3) / 1e12
     step_tf = (mask_flops + attn_flops) / (total_ms * 1e-3 / steps) / 1e12
-    launches_per_step = 2  # hip_mask + hip_sparse_attn (the split merge is fused)
+    # hip_mask + hip_sparse_attn (their split merge is fused), or one launch
+    launches_per_step = 1 if one_launch else 2
+    two_call = None
+    if fused:
+        # the same step as the two separate calls, for comparison (not timed above)
+        ev2 = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * layers)]
+        g3 = graph_with_events(ev2, False)
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, min(50, reps))):
+                g3.replay()
+        stream.synchronize()
+        sess.check()
+        m2 = np.mean([ev2[3 * l].elapsed_time(ev2[3 * l + 1]) for l in range(layers)])
+        a2 = np.mean([ev2[3 * l + 1].elapsed_time(ev2[3 * l + 2]) for l in range(layers)])
+        two_call = {"mask_us": m2 * 1e3, "attn_us": a2 * 1e3, "step_us": (m2 + a2) * 1e3,
+                    "how": "hip_mask + hip_sparse_attn, CUDA event nodes, last of up to 50 replays"}
+        del g3
 
     # e2e: per step, H2D of the step's query and new key/value rows from pinned
     # host memory, the two C-ABI calls, D2H of the output; captured as a graph
@@ -516,8 +557,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
             qs[l].copy_(hq[l], non_blocking=True)
             ks[l][:, :, w.seq_len - 1].copy_(krow, non_blocking=True)
             vs[l][:, :, w.seq_len - 1].copy_(vrow, non_blocking=True)
-            hb.hip_mask(qs[l], ks[l], sess.p, idxs[l])
-            hb.hip_sparse_attn(qs[l], ks[l], vs[l], idxs[l], sess.p, outs[l])
+            step(l)
             hout[l].copy_(outs[l], non_blocking=True)
 
         g2 = torch.cuda.CUDAGraph()
@@ -549,7 +589,9 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         h2d = (q0.numel() + krow.numel() + vrow.numel()) * esz
         e2e = {"value": whole_job_us_per_layer(e2e_ms, steps, world), "unit": "us/layer",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(q0.numel() * esz),
-               "how": "CUDA graph of H2D (pinned) + hip_mask + hip_sparse_attn + D2H per step"}
+               "how": "CUDA graph per step: H2D (pinned) of q and the new k/v row, "
+                      + ("hip_mask_sparse_attn" if fused else "hip_mask + hip_sparse_attn")
+                      + ", D2H of out"}
         sess.check()
 
     if not args.no_e2e and prefill:
@@ -597,10 +639,19 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
                     "algorithmic_flops": attn_flops if dom_attn else mask_flops}
         value, unit, hib = step_tf, "TFLOP/s", True
     else:
-        roofline = {"bound": "hbm", "kernel": mask_kernel, "achieved": mask_gbs,
-                    "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s", "frac": mask_gbs / hbm,
-                    "traffic": traffic_from_profile(mask_kernel, w.name),
-                    "algorithmic_bytes": mask_bytes}
+        if one_launch:
+            # one kernel does the whole step: its bytes are the mask's and the attention's
+            fused_gbs = (mask_bytes + attn_bytes) / (mask_ms * 1e-3) / 1e9
+            roofline = {"bound": "hbm", "kernel": mask_kernel + " (mask + attention)",
+                        "achieved": fused_gbs, "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s",
+                        "frac": fused_gbs / hbm,
+                        "traffic": traffic_from_profile(mask_kernel + "+attn", w.name),
+                        "algorithmic_bytes": mask_bytes + attn_bytes}
+        else:
+            roofline = {"bound": "hbm", "kernel": mask_kernel, "achieved": mask_gbs,
+                        "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s", "frac": mask_gbs / hbm,
+                        "traffic": traffic_from_profile(mask_kernel, w.name),
+                        "algorithmic_bytes": mask_bytes}
         value, unit, hib = us_layer, "us/layer", False
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
@@ -613,7 +664,9 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": step_gbs / hbm, "algorithmic_bytes": mask_bytes + attn_bytes},
         "kernels": {"how": "CUDA event nodes around each call, last full graph replay of the timed region",
-                    "mask_kernel": mask_kernel, "attn_kernel": attn_kernel,
+                    "step_call": "hip_mask_sparse_attn" if fused else "hip_mask + hip_sparse_attn",
+                    "one_launch": one_launch,
+                    "mask_kernel": mask_kernel, "attn_kernel": None if one_launch else attn_kernel,
                     "mask_us": mask_ms * 1e3, "mask_bytes": mask_bytes, "mask_gbs": mask_gbs,
                     "mask_tflops": mask_tf, "mask_flops": mask_flops, "scored_candidates": scored,
                     "attn_us": attn_ms * 1e3, "attn_bytes": attn_bytes, "attn_gbs": attn_gbs,
@@ -621,6 +674,8 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         "gpu_launches": launches_per_step * steps,
         "clocks": clk.summary(),
     }
+    if two_call:
+        line["kernels"]["two_calls"] = two_call
     if prefill:
         line["step_tflops"] = step_tf
         line["us_per_layer"] = us_layer

@@ -25,10 +25,12 @@ HIPS_BF16 = 1
 OP_MASK = 0
 OP_SPARSE = 1
 OP_DENSE = 2
+OP_MASK_SPARSE = 3
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhip_sparse.so")
 EXPORTS = ("hip_idx_row_stride", "hip_workspace_size", "hip_workspace_init", "hip_check_status",
-           "hip_mask", "hip_sparse_attn", "hip_dense_attn", "hip_last_cuda_error",
+           "hip_mask", "hip_sparse_attn", "hip_mask_sparse_attn", "hip_dense_attn",
+           "hip_sparse_attn_noalloc", "hip_last_cuda_error",
            "hip_error_string")
 
 
@@ -81,6 +83,8 @@ def load() -> ctypes.CDLL:
     lib.hip_mask.argtypes = [vp, vp, P, vp]
     lib.hip_sparse_attn.restype = ctypes.c_int
     lib.hip_sparse_attn.argtypes = [vp, vp, vp, vp, P, vp]
+    lib.hip_mask_sparse_attn.restype = ctypes.c_int
+    lib.hip_mask_sparse_attn.argtypes = [vp, vp, vp, P, vp, vp]
     lib.hip_dense_attn.restype = ctypes.c_int
     lib.hip_dense_attn.argtypes = [vp, vp, vp, P, vp]
     lib.hip_sparse_attn_noalloc.restype = ctypes.c_int
@@ -141,6 +145,11 @@ def sparse_attn_ptr(q: int, k: int, v: int, idx: int, p: Params, out: int) -> in
                                       ctypes.byref(p), out or None))
 
 
+def mask_sparse_attn_ptr(q: int, k: int, v: int, p: Params, idx_out: int, out: int) -> int:
+    return int(load().hip_mask_sparse_attn(q or None, k or None, v or None, ctypes.byref(p),
+                                           idx_out or None, out or None))
+
+
 def sparse_attn_noalloc_ptr(q: int, k: int, v: int, idx: int, p: Params, out: int) -> int:
     """hip_sparse_attn on the library's fixed scratch array (no workspace)."""
     return int(load().hip_sparse_attn_noalloc(q or None, k or None, v or None, idx or None,
@@ -179,6 +188,12 @@ def hip_sparse_attn(q, k, v, idx, p: Params, out) -> None:
     _check("hip_sparse_attn", sparse_attn_ptr(_dev(q), _dev(k), _dev(v), _dev(idx), p, _dev(out)))
 
 
+def hip_mask_sparse_attn(q, k, v, p: Params, idx_out, out) -> None:
+    """hip_mask then hip_sparse_attn on its idx (one launch for decode shapes)."""
+    _check("hip_mask_sparse_attn",
+           mask_sparse_attn_ptr(_dev(q), _dev(k), _dev(v), p, _dev(idx_out), _dev(out)))
+
+
 def hip_sparse_attn_noalloc(q, k, v, idx, p: Params, out) -> None:
     """Sparse attention for callers that cannot allocate device memory: the
     split-K scratch is a fixed array inside the library (see the header)."""
@@ -208,7 +223,7 @@ class Session:
                         block_k=block_k, topk=topk, sink=sink, window=window,
                         mask_len=mask_len, kv_capacity=kv_capacity,
                         stream=self.stream.cuda_stream)
-        need = max(workspace_size(self.p, op) for op in (OP_MASK, OP_SPARSE, OP_DENSE))
+        need = max(workspace_size(self.p, op) for op in (OP_MASK, OP_SPARSE, OP_DENSE, OP_MASK_SPARSE))
         if need == 0:
             raise HipsError("hip_workspace_size", HIPS_ERR_INVALID_ARG, "invalid parameters")
         self.workspace = torch.empty(need + 256, dtype=torch.uint8, device="cuda")
@@ -223,7 +238,7 @@ class Session:
         """Change scalar fields (seq_len, mask_len, q_pos0 ...) in place."""
         for key, val in kw.items():
             setattr(self.p, key, val)
-        need = max(workspace_size(self.p, op) for op in (OP_MASK, OP_SPARSE, OP_DENSE))
+        need = max(workspace_size(self.p, op) for op in (OP_MASK, OP_SPARSE, OP_DENSE, OP_MASK_SPARSE))
         if need > self.p.workspace_bytes:
             raise HipsError("hip_workspace_size", HIPS_ERR_WORKSPACE, "workspace too small")
         self.row_stride = idx_row_stride(self.p)
@@ -243,6 +258,14 @@ class Session:
         o = torch.empty_like(q) if out is None else out
         hip_sparse_attn(q, k, v, idx, self.p, o)
         return o
+
+    def mask_sparse_attn(self, q, k, v, idx_out=None, out=None):
+        """Fresh mask and attention over it; returns (idx, out)."""
+        import torch
+        idx = self.new_idx() if idx_out is None else idx_out
+        o = torch.empty_like(q) if out is None else out
+        hip_mask_sparse_attn(q, k, v, self.p, idx, o)
+        return idx, o
 
     def dense_attn(self, q, k, v, out=None):
         import torch

@@ -283,6 +283,55 @@ int run_attention(const void* q, const void* k, const void* v, const int32_t* id
                               : hips::launch_attn_fma(a, plan.smem, stream));
 }
 
+// The tensor-core mask kernel also runs the attention of its mask row (one
+// launch for a decode step) when the row group is a single MMA column block
+// of at most mask_mma_fused_rows() query rows.
+bool fusable(const MaskPlan& plan) {
+  return plan.mma && hips::mask_mma_nc(plan.a.rows_max) == 1 &&
+         plan.a.rows_max <= hips::mask_mma_fused_rows();
+}
+
+// Plan and launch the mask kernel (with the fused attention when v and out
+// are given). A cluster of C CTAs needs C free SMs of one GPC: take the
+// largest cluster for which every mask row is resident at once (one wave);
+// fall back to smaller clusters if the device refuses the shape.
+int launch_mask(const void* q, const void* k, const hips_params* params, int32_t* idx_out,
+                const void* v, void* out) {
+  MaskPlan plan;
+  int st = plan_mask(params, 16, &plan);
+  if (st) return st;
+  st = check_workspace(params, plan.ws);
+  if (st) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
+  for (int cap = 16; cap >= 1; cap = std::min(cap - 1, plan.a.cluster - 1)) {
+    st = plan_mask(params, cap, &plan);
+    if (st) return st;
+    if (plan.a.cluster > cap) continue;
+    if (plan.a.cluster > 1 && cap > 1) {
+      const int fit = resident_clusters(plan);
+      if (fit >= 0 && fit < plan.a.units) continue;
+    }
+    hips::MaskArgs& a = plan.a;
+    a.q = q; a.k = k; a.idx = idx_out;
+    a.status = static_cast<hips::Status*>(params->workspace);
+    if (out) {
+      if (!fusable(plan)) return HIPS_ERR_UNSUPPORTED;
+      a.v = v;
+      a.out = out;
+      a.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
+    }
+    const cudaError_t e = plan.mma ? hips::launch_mask_mma(a, plan.smem, stream)
+                                   : hips::launch_mask_fma(a, plan.smem, stream);
+    if (e == cudaSuccess) return HIPS_OK;
+    if ((e == cudaErrorInvalidClusterSize || e == cudaErrorLaunchOutOfResources) && cap > 1) {
+      (void)cudaGetLastError();
+      continue;
+    }
+    return cuda_status(e);
+  }
+  return HIPS_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 namespace hips {
@@ -326,6 +375,11 @@ size_t hip_workspace_size(const hips_params* params, int op) {
     MaskPlan plan;
     return plan_mask(params, 16, &plan) == HIPS_OK ? plan.ws : 0;
   }
+  if (op == HIPS_OP_MASK_SPARSE) {  // either the fused launch or the two calls
+    const size_t m = hip_workspace_size(params, HIPS_OP_MASK);
+    const size_t s = hip_workspace_size(params, HIPS_OP_SPARSE);
+    return m && s ? std::max(m, s) : 0;
+  }
   if (op == HIPS_OP_SPARSE || op == HIPS_OP_DENSE) {
     AttnPlan plan;
     return plan_attn(params, op == HIPS_OP_DENSE, &plan) == HIPS_OK ? plan.ws : 0;
@@ -358,36 +412,25 @@ int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* i
   if (st) return st;
   if (!q || !k || !idx_out) return HIPS_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx_out, 4)) return HIPS_ERR_INVALID_ARG;
+  return launch_mask(q, k, params, idx_out, nullptr, nullptr);
+}
+
+int hip_mask_sparse_attn(const void* q, const void* k, const void* v, const hips_params* params,
+                         int32_t* idx_out, void* out) {
+  int st = validate(params, HIPS_OP_MASK_SPARSE);
+  if (st) return st;
+  if (!q || !k || !v || !idx_out || !out) return HIPS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(idx_out, 4))
+    return HIPS_ERR_INVALID_ARG;
+  if (params->mask_len != params->seq_len) return HIPS_ERR_INVALID_ARG;  // a fresh mask
   MaskPlan plan;
   st = plan_mask(params, 16, &plan);
   if (st) return st;
-  st = check_workspace(params, plan.ws);
+  if (fusable(plan)) return launch_mask(q, k, params, idx_out, v, out);
+  st = launch_mask(q, k, params, idx_out, nullptr, nullptr);
   if (st) return st;
-  cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
-  // A cluster of C CTAs needs C free SMs of one GPC. Take the largest cluster
-  // for which every mask row is resident at once (one wave); fall back to
-  // smaller clusters if the device refuses the shape.
-  for (int cap = 16; cap >= 1; cap = std::min(cap - 1, plan.a.cluster - 1)) {
-    st = plan_mask(params, cap, &plan);
-    if (st) return st;
-    if (plan.a.cluster > cap) continue;
-    if (plan.a.cluster > 1 && cap > 1) {
-      const int fit = resident_clusters(plan);
-      if (fit >= 0 && fit < plan.a.units) continue;
-    }
-    hips::MaskArgs& a = plan.a;
-    a.q = q; a.k = k; a.idx = idx_out;
-    a.status = static_cast<hips::Status*>(params->workspace);
-    const cudaError_t e = plan.mma ? hips::launch_mask_mma(a, plan.smem, stream)
-                                   : hips::launch_mask_fma(a, plan.smem, stream);
-    if (e == cudaSuccess) return HIPS_OK;
-    if ((e == cudaErrorInvalidClusterSize || e == cudaErrorLaunchOutOfResources) && cap > 1) {
-      (void)cudaGetLastError();
-      continue;
-    }
-    return cuda_status(e);
-  }
-  return HIPS_ERR_UNSUPPORTED;
+  return run_attention(q, k, v, idx_out, params, out, false);
 }
 
 int hip_sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx,

@@ -18,6 +18,11 @@ struct MaskArgs {
   int dtype, n_qheads, n_kvheads, group, q_len, block_q, block_k, n0max, sink, window;
   int nqb, cluster, per_cta, rows_max, rows_pad, stages;
   int64_t units, seq_len, kv_cap, q_pos0, row_stride;
+  // fused decode (tensor-core mask, few rows): when out is set, the cluster
+  // of a mask row also computes the row's sparse attention over v
+  const void* v;
+  void* out;
+  float scale_log2;
 };
 
 struct AttnArgs {
@@ -49,6 +54,7 @@ int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster);
 int mask_mma_tile_keys();
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream);
+int mask_mma_fused_rows();  // most query rows of a fused mask + attention launch
 
 // Tensor-core attention for query blocks, bf16 (attn_mma.cu)
 int attn_mma_smem_bytes(int table_items);

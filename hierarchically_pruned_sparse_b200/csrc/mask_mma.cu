@@ -39,6 +39,8 @@
 //    with t_r + eps_r < max_r' (t_r' - eps_r') has s_r < s.
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "hips_common.cuh"
 #include "hips_kernels.h"
 #include "hips_tc.cuh"
@@ -85,7 +87,7 @@ __host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cl
   int o = 0;
   L.ring = o;     o += S * kTileBytes;
   L.bq = o;       o += nc * 16 * 256;
-  L.bar = o;      o += 8 * (2 * S + 5);
+  L.bar = o;      o += 8 * (3 * S + 5);
   L.slot = o;     o += 16;
   L.rpos = o;     o += nc * 16 * 4;  // query position offset (r % b_q) of operand row r
   L.qn = o;       o += nc * 16 * 4;  // |q_r|_2, rounded up (0 for padding rows)
@@ -270,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   uint64_t* mma_done = empty + S;    // [2]: accumulator written
   uint64_t* tm_empty = mma_done + 2; // [2]: accumulator read back
   uint64_t* band_bar = tm_empty + 2; // band MMA done
+  uint64_t* abar = band_bar + 1;     // [S]: attention tile landed (fused decode)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.slot);
   int* rpos = reinterpret_cast<int*>(smem + L.rpos);
   float* qn = reinterpret_cast<float*>(smem + L.qn);
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       mbar_init(&tm_empty[s], 4);
     }
     mbar_init(band_bar, 1);
+    for (int s = 0; s < S; ++s) mbar_init(&abar[s], kThreads);
     fence_mbar_init();
   }
   __syncwarp();
@@ -803,38 +807,271 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   // ascending) is the kept set
   const int* chunk_s = cs_all + cur * nbuf;
 
-  // ---- union with sink and window blocks, write the idx row (CTA 0)
-  if (rank == 0) {
-    const int64_t ns = min64((a.sink + bk - 1) / bk, N_blocks);
-    const int64_t cutb = a.window > 0 ? max64(0, q_first - a.window + 1) / bk : N_blocks;
-    const int64_t lead = min64(ns, cutb);
-    int lo_i = 0, hi_i = n0;
-    {
-      int l = 0, h = n0;
-      while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < ns) l = m + 1; else h = m; }
-      lo_i = l;
-      l = lo_i; h = n0;
-      while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < cutb) l = m + 1; else h = m; }
-      hi_i = l;
+  // ---- union with sink and window blocks: the idx row is the sink blocks
+  // [0, lead), the kept chunks chunk_s[lo_i, lo_i + mid), then the window
+  // blocks [cutb, N_blocks)
+  const int64_t ns = min64((a.sink + bk - 1) / bk, N_blocks);
+  const int64_t cutb = a.window > 0 ? max64(0, q_first - a.window + 1) / bk : N_blocks;
+  const int64_t lead = min64(ns, cutb);
+  int lo_i = 0, hi_i = n0;
+  {
+    int l = 0, h = n0;
+    while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < ns) l = m + 1; else h = m; }
+    lo_i = l;
+    l = lo_i; h = n0;
+    while (l < h) { const int m = (l + h) / 2; if (chunk_s[m] < cutb) l = m + 1; else h = m; }
+    hi_i = l;
+  }
+  const int64_t mid = hi_i > lo_i ? hi_i - lo_i : 0;
+  const int64_t tail = a.window > 0 ? N_blocks - cutb : 0;
+  const int64_t nnz = lead + mid + tail;
+  auto block_at = [&](int64_t e) -> int64_t {
+    return e < lead ? e : (e < lead + mid ? chunk_s[lo_i + (e - lead)] : cutb + (e - lead - mid));
+  };
+  auto write_idx = [&]() {
+    if (rank == 0) {
+      int32_t* row = a.idx + unit * a.row_stride;
+      for (int64_t t = tid; t < a.row_stride; t += kThreads)
+        row[t] = static_cast<int32_t>(t == 0 ? nnz : (t - 1 < nnz ? block_at(t - 1) : -1));
     }
-    const int64_t mid = hi_i > lo_i ? hi_i - lo_i : 0;
-    const int64_t tail = a.window > 0 ? N_blocks - cutb : 0;
-    const int64_t nnz = lead + mid + tail;
-    int32_t* row = a.idx + unit * a.row_stride;
-    for (int64_t t = tid; t < a.row_stride; t += kThreads) {
-      int64_t val;
-      if (t == 0) {
-        val = nnz;
-      } else {
-        const int64_t e = t - 1;
-        if (e < lead) val = e;
-        else if (e < lead + mid) val = chunk_s[lo_i + (e - lead)];
-        else if (e < nnz) val = cutb + (e - lead - mid);
-        else val = -1;
-      }
-      row[t] = static_cast<int32_t>(val);
+  };
+  bool idx_written = false;
+
+  if constexpr (NC == 1) {
+    if (a.out != nullptr) {
+      // ---- fused decode: the cluster attends the row's blocks right away.
+      // CTA `rank` takes a contiguous share of the idx row; its K and V rows
+      // go through the (now idle) ring in 64-key tiles; 8 lanes per key, two
+      // keys per 8-lane group and tile; fp32 online softmax in the exp2
+      // domain with the reference max moved only when a score exceeds it by
+      // more than 2^8; the group, warp and CTA partials are then merged, the
+      // last across the cluster by CTA 0 through distributed shared memory.
+      auto fused = [&](auto rc_tag) {
+        constexpr int RC = decltype(rc_tag)::value;
+        constexpr int kAK = 64;  // keys per attention tile
+        const int64_t ipc = (nnz + C - 1) / C;
+        const int64_t it0 = min64(nnz, rank * ipc), it1 = min64(nnz, it0 + ipc);
+        const int ipt = kAK >> lbk;
+        const int ntl = static_cast<int>((it1 - it0 + ipt - 1) / ipt);
+        const unsigned char* vbase = static_cast<const unsigned char*>(a.v) +
+                                     (static_cast<int64_t>(b) * a.n_kvheads + g) * a.kv_cap * 256;
+        auto issue = [&](int t) {
+          const int slot = t % S;
+          unsigned char* kd = ring + slot * kTileBytes;
+          unsigned char* vd = kd + kHalfBytes;
+          const int64_t f = it0 + static_cast<int64_t>(t) * ipt;
+          const int nk = static_cast<int>(min64(ipt, it1 - f)) << lbk;
+          for (int i = tid; i < nk * 16; i += kThreads) {
+            const int kk = i >> 4, ch = i & 15;
+            const int64_t j = (block_at(f + (kk >> lbk)) << lbk) + (kk & (bk - 1));
+            if (j < Tc) {
+              cp_async16(kd + kk * 256 + ch * 16, kbase + j * 256 + ch * 16);
+              cp_async16(vd + kk * 256 + ch * 16, vbase + j * 256 + ch * 16);
+            }
+          }
+          cp_async_arrive(&abar[slot]);
+        };
+        for (int t = 0; t < min(S, ntl); ++t) issue(t);
+        write_idx();  // while the first tiles are on their way
+        idx_written = true;
+
+        float qreg[RC][16];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) {
+          if (r < R) {
+            const int h = g * a.group + r / nrows, qi = i0 + r % nrows;
+            load_row16<uint16_t>(reinterpret_cast<const unsigned char*>(
+                                     qg + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + qi) * kD),
+                                 lane8, qreg[r]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) qreg[r][e] = 0.0f;
+          }
+        }
+        int plim[RC];  // last key position row r sees
+#pragma unroll
+        for (int r = 0; r < RC; ++r) plim[r] = r < R ? static_cast<int>(q_first + rpos[r]) : -1;
+        float mref[RC], lsum[RC], o[RC][16];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) {
+          mref[r] = -INFINITY;
+          lsum[r] = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[r][e] = 0.0f;
+        }
+        for (int t = 0; t < ntl; ++t) {
+          const int slot = t % S;
+          if (!timed_out && !mbar_wait(&abar[slot], (t / S) & 1)) timed_out = true;
+          const int64_t f = it0 + static_cast<int64_t>(t) * ipt;
+          const int nk = static_cast<int>(min64(ipt, it1 - f)) << lbk;
+          const unsigned char* kt = ring + slot * kTileBytes;
+          const unsigned char* vt = kt + kHalfBytes;
+          // this group's two keys of the tile: scores of both keys and every
+          // row first (independent chains), then one reference-max check
+          int64_t jj[2];
+          float kx[2][16], vx[2][16];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int kk = warp * 8 + grp + 4 * u;
+            jj[u] = -1;
+            if (kk < nk) {
+              const int64_t j = (block_at(f + (kk >> lbk)) << lbk) + (kk & (bk - 1));
+              jj[u] = j < Tc ? j : -1;
+            }
+            load_row16<uint16_t>(kt + kk * 256, lane8, kx[u]);
+            load_row16<uint16_t>(vt + kk * 256, lane8, vx[u]);
+          }
+          float sc[2][RC];
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+              float d0 = 0.0f, d1 = 0.0f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                d0 = fmaf(qreg[r][e], kx[u][e], d0);
+                d1 = fmaf(qreg[r][8 + e], kx[u][8 + e], d1);
+              }
+              sc[u][r] = d0 + d1;
+            }
+#pragma unroll
+          for (int o_ = 4; o_; o_ >>= 1)
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+              for (int r = 0; r < RC; ++r) sc[u][r] += __shfl_xor_sync(0xffffffffu, sc[u][r], o_);
+          bool grow = false;
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+              sc[u][r] = (jj[u] >= 0 && jj[u] <= plim[r]) ? sc[u][r] * a.scale_log2 : -INFINITY;
+              grow |= sc[u][r] > mref[r] + 8.0f;
+            }
+          if (__any_sync(0xffffffffu, grow)) {  // rare: move the reference max
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+              const float smax = fmaxf(sc[0][r], sc[1][r]);
+              if (smax > mref[r] + 8.0f) {
+                const float al = mref[r] == -INFINITY ? 0.0f : exp2f(mref[r] - smax);
+                lsum[r] *= al;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) o[r][e] *= al;
+                mref[r] = smax;
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+              const float pk = sc[u][r] == -INFINITY ? 0.0f : exp2f(sc[u][r] - mref[r]);
+              lsum[r] += pk;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[r][e] = fmaf(pk, vx[u][e], o[r][e]);
+            }
+          __syncthreads();  // every warp is done with this slot
+          if (t + S < ntl) issue(t + S);
+        }
+        // merge the 4 groups of a warp
+#pragma unroll
+        for (int off = 8; off <= 16; off <<= 1) {
+#pragma unroll
+          for (int r = 0; r < RC; ++r) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, mref[r], off);
+            const float l2 = __shfl_xor_sync(0xffffffffu, lsum[r], off);
+            const float mm = fmaxf(mref[r], m2);
+            const float a1 = mref[r] == -INFINITY ? 0.0f : exp2f(mref[r] - mm);
+            const float a2 = m2 == -INFINITY ? 0.0f : exp2f(m2 - mm);
+            lsum[r] = lsum[r] * a1 + l2 * a2;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float o2 = __shfl_xor_sync(0xffffffffu, o[r][e], off);
+              o[r][e] = o[r][e] * a1 + o2 * a2;
+            }
+            mref[r] = mm;
+          }
+        }
+        // warp partials -> CTA partial (ring: [warp][row][m, l, pad, pad, o[128]])
+        constexpr int kPS = kD + 4;
+        float* wpart = reinterpret_cast<float*>(ring);
+        float* cpart = reinterpret_cast<float*>(ring + 32768);  // [row][kPS]
+        if (grp == 0) {
+#pragma unroll
+          for (int r = 0; r < RC; ++r) {
+            float* w = wpart + (warp * RC + r) * kPS;
+            if (lane8 == 0) {
+              w[0] = mref[r];
+              w[1] = lsum[r];
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              w[4 + lane8 * 8 + e] = o[r][e];
+              w[4 + 64 + lane8 * 8 + e] = o[r][8 + e];
+            }
+          }
+        }
+        __syncthreads();
+        for (int x = tid; x < R * kD; x += kThreads) {
+          const int r = x >> 7, e = x & (kD - 1);
+          float mm = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, wpart[(w * RC + r) * kPS]);
+          float l = 0.0f, ov = 0.0f;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const float* wp = wpart + (w * RC + r) * kPS;
+            const float sc = wp[0] == -INFINITY ? 0.0f : exp2f(wp[0] - mm);
+            l += wp[1] * sc;
+            ov += wp[4 + e] * sc;
+          }
+          if (e == 0) {
+            cpart[r * kPS] = mm;
+            cpart[r * kPS + 1] = l;
+          }
+          cpart[r * kPS + 4 + e] = ov;
+        }
+        if (C > 1) cluster.sync();  // every CTA's partial is ready
+        else __syncthreads();
+        // CTA `rank` merges the C partials of head dims [rank * dpc, +dpc):
+        // all remote loads first (one round trip), then the merge
+        const int dpc = (kD + C - 1) / C;
+        for (int x = tid; x < R * dpc; x += kThreads) {
+          const int r = x / dpc, e = rank * dpc + (x - r * dpc);
+          if (e >= kD) continue;
+          float mv[16], lv[16], ov[16];
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            mv[p] = -INFINITY;
+            lv[p] = 0.0f;
+            ov[p] = 0.0f;
+            if (p < C) {
+              const float* cp = C > 1 ? cluster.map_shared_rank(cpart, p) : cpart;
+              mv[p] = cp[r * kPS];
+              lv[p] = cp[r * kPS + 1];
+              ov[p] = cp[r * kPS + 4 + e];
+            }
+          }
+          float mm = -INFINITY;
+#pragma unroll
+          for (int p = 0; p < 16; ++p) mm = fmaxf(mm, mv[p]);
+          float l = 0.0f, o_sum = 0.0f;
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const float sc = mv[p] == -INFINITY ? 0.0f : exp2f(mv[p] - mm);
+            l += lv[p] * sc;
+            o_sum += ov[p] * sc;
+          }
+          const int h = g * a.group + r / nrows, qi = i0 + r % nrows;
+          uint16_t* orow = static_cast<uint16_t*>(a.out) +
+                           ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + qi) * kD;
+          orow[e] = f2bf16_rn(l > 0.0f ? o_sum / l : 0.0f);
+        }
+      };
+      fused(std::integral_constant<int, 4>{});  // the planner keeps R <= mask_mma_fused_rows()
     }
   }
+  if (!idx_written) write_idx();
   if (timed_out) report(a.status, kStatusTimeout, 3);
   tc_fence_before_sync();
   __syncthreads();
@@ -918,6 +1155,8 @@ int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster) {
 }
 
 int mask_mma_tile_keys() { return kM; }
+
+int mask_mma_fused_rows() { return 4; }
 
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem) {
   switch (mask_mma_nc(a.rows_max)) {

@@ -80,7 +80,7 @@ enum hips_status {
 
 enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1 };
 
-enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2 };
+enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2, HIPS_OP_MASK_SPARSE = 3 };
 
 typedef struct hips_params {
   int32_t batch;      /* sequences */
@@ -129,6 +129,20 @@ HIPS_API int hip_mask(const void* q, const void* k, const hips_params* params, i
  * plus the keys [mask_len, seq_len). out: [B, Hq, q_len, d] in dtype. */
 HIPS_API int hip_sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx,
                     const hips_params* params, void* out);
+
+/* hip_mask followed by hip_sparse_attn on its idx, for a freshly computed
+ * mask (mask_len must equal seq_len, else HIPS_ERR_INVALID_ARG): writes
+ * idx_out exactly as hip_mask does and out as hip_sparse_attn does. For
+ * decode-shaped groups (at most 4 query rows per mask row, bf16) one launch
+ * does both: the thread-block cluster that selects a row's blocks then
+ * attends over them, each CTA over a contiguous share of the row, and the
+ * CTAs' partial softmax sums are merged through distributed shared memory.
+ * Other shapes run the two calls. Workspace: hip_workspace_size(params,
+ * HIPS_OP_MASK_SPARSE). This is the sequence of the two steps defined above,
+ * (Author Rebuttal to the Reviewer RsGC, Q2, then Reviewer NLBm, W2), in one
+ * call. */
+HIPS_API int hip_mask_sparse_attn(const void* q, const void* k, const void* v,
+                                  const hips_params* params, int32_t* idx_out, void* out);
 
 /* Dense causal attention over keys [0, seq_len); block/topk fields ignored. */
 HIPS_API int hip_dense_attn(const void* q, const void* k, const void* v, const hips_params* params,

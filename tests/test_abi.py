@@ -77,7 +77,9 @@ def test_bad_arguments_rejected_on_host(bad, code):
     fake = 1 << 20  # never dereferenced: validation fails first
     assert hb.mask_ptr(fake, fake, p, fake) == code
     assert hb.sparse_attn_ptr(fake, fake, fake, fake, p, fake) == code
+    assert hb.mask_sparse_attn_ptr(fake, fake, fake, p, fake, fake) == code
     assert hb.workspace_size(p, hb.OP_MASK) == 0
+    assert hb.workspace_size(p, hb.OP_MASK_SPARSE) == 0
 
 
 def test_null_and_misaligned_pointers_rejected():
@@ -100,6 +102,21 @@ def test_workspace_checked_before_launch():
     assert hb.sparse_attn_ptr(f, f, f, f, p, f) == hb.HIPS_ERR_WORKSPACE
     p = _decode_params(workspace=f + 16, workspace_bytes=need)  # not 256-byte aligned
     assert hb.sparse_attn_ptr(f, f, f, f, p, f) == hb.HIPS_ERR_WORKSPACE
+
+
+def test_fused_call_checks_on_host():
+    f = 1 << 20
+    need = hb.workspace_size(_decode_params(), hb.OP_MASK_SPARSE)
+    assert need == max(hb.workspace_size(_decode_params(), hb.OP_MASK),
+                       hb.workspace_size(_decode_params(), hb.OP_SPARSE))
+    # a reused mask (keys appended since it was computed) is not a fresh mask
+    p = _decode_params(seq_len=131080, kv_capacity=131080, q_pos0=131079, mask_len=131072,
+                       workspace=f, workspace_bytes=need)
+    assert hb.mask_sparse_attn_ptr(f, f, f, p, f, f) == hb.HIPS_ERR_INVALID_ARG
+    p = _decode_params(workspace=f, workspace_bytes=need)
+    assert hb.mask_sparse_attn_ptr(f, f, 0, p, f, f) == hb.HIPS_ERR_INVALID_ARG   # v missing
+    assert hb.mask_sparse_attn_ptr(f, f, f, p, f, f + 8) == hb.HIPS_ERR_INVALID_ARG  # out misaligned
+    assert hb.mask_sparse_attn_ptr(f, f, f, _decode_params(), f, f) == hb.HIPS_ERR_WORKSPACE
 
 
 def test_prefill_shapes_plan():

@@ -97,6 +97,32 @@ def test_small_decode(w):
     _check(w)
 
 
+FUSED = SMALL + [W.DECODE_128K]
+
+
+@pytest.mark.parametrize("w", FUSED, ids=[w.name for w in FUSED])
+def test_mask_then_attention_in_one_call(w):
+    """hip_mask_sparse_attn: the same idx as hip_mask, and attention within
+    tolerance of the oracle (one launch for bf16 groups of <= 4 rows, the two
+    calls otherwise)."""
+    import torch
+    x = _inputs(w)
+    osh, bkw = pu.shapes(w)
+    q, k, v = pu.torch_inputs(x, w)
+    s = _session(bkw)
+    idx_f, out_f = s.mask_sparse_attn(q, k, v)
+    idx_m = s.mask(q, k)
+    torch.cuda.synchronize()
+    s.check()
+    idx_f = idx_f.cpu().numpy()
+    assert np.array_equal(idx_f, idx_m.cpu().numpy())
+    idx_ref, gap, _ = oracle.mask(x["q"][0], x["k"], osh)
+    st = pu.compare_masks(idx_f.reshape(idx_ref.shape), idx_ref, gap)
+    if st["mismatched"] == 0:
+        ref = oracle.attention(x["q"][0], x["k"], x["v"], idx_ref, osh)
+        pu.compare_outputs(out_f.float().cpu().numpy().reshape(ref.shape), ref, w.dtype)
+
+
 def test_decode_8k_f32():
     st = _check(W.DECODE_8K_F32)
     assert st["mismatched"] == 0
