@@ -82,21 +82,21 @@ __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
 // into every CTA of the cluster; two copies alternate between rounds.
 __host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cluster) {
   MmaSmem L;
-  const int n = 2 * n0max;
+  const int n = (2 * n0max + 3) & ~3;  // candidate buffer stride (16-byte rows of 4)
   const int S = stages_for(nc, per);
   int o = 0;
   L.ring = o;     o += S * kTileBytes;
   L.bq = o;       o += nc * 16 * 256;
-  L.bar = o;      o += 8 * (3 * S + 5);
+  L.bar = o;      o += al(8 * (3 * S + 5), 16);  // every region below starts on 16 bytes
   L.slot = o;     o += 16;
   L.rpos = o;     o += nc * 16 * 4;  // query position offset (r % b_q) of operand row r
   L.qn = o;       o += nc * 16 * 4;  // |q_r|_2, rounded up (0 for padding rows)
-  L.cs = o;       o += 2 * al(n * 4, 16);
-  L.ce = o;       o += 2 * al(n * 4, 16);
+  L.cs = o;       o += 2 * n * 4;
+  L.ce = o;       o += 2 * n * 4;
   L.keepb = o;    o += al(n, 16);
-  L.band = o;     o += al(n * 4, 16);
-  L.band_key = o; o += al(n * 4, 16);
-  L.xch = o;      o += (cluster > 1 ? 2 : 1) * al(n * 8, 16);
+  L.band = o;     o += n * 4;
+  L.band_key = o; o += n * 4;
+  L.xch = o;      o += (cluster > 1 ? 2 : 1) * n * 8;
   L.hist = o;     o += kBuckets * 4;
   L.rowmask = o;  o += nc >= 4 ? kM * mask_words(nc) * 4 : 0;
   L.scratch = o;  o += 64 * 4;
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   const int64_t N_blocks = (Tc + bk - 1) / bk;
   const int n0 = static_cast<int>(min64(a.n0max, N_blocks));
   const int per_cta = a.per_cta;
-  const int nbuf = 2 * a.n0max;  // stride between the two candidate buffers
+  const int nbuf = (2 * a.n0max + 3) & ~3;  // stride between the two candidate buffers
 
   const MmaSmem L = mma_layout(NC, PER, a.n0max, C);
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -503,13 +503,15 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     tc_fence_after_sync();
     if (C > 1) cluster.sync();
     float tv[PER], ev[PER];
-    const int ibase = tid * PER;
+    const int ibase = tid * PER;  // 16-byte vector loads of this thread's entries
 #pragma unroll
-    for (int q = 0; q < PER; ++q) {
-      const int i = ibase + q;
-      const float2 x = i < ncand ? my_x[i] : make_float2(0.0f, 0.0f);
-      tv[q] = x.x;
-      ev[q] = x.y;
+    for (int v = 0; v < PER / 2; ++v) {
+      float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (ibase + 2 * v < ncand) x = reinterpret_cast<const float4*>(my_x + ibase)[v];
+      tv[2 * v] = x.x;
+      ev[2 * v] = x.y;
+      tv[2 * v + 1] = x.z;
+      ev[2 * v + 1] = x.w;
     }
     float lo = INFINITY, hi = -INFINITY, emax = 0.0f;
 #pragma unroll
@@ -594,7 +596,11 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         const float t = tv[q], e = ev[q];
         cl[q] = t - e > upper ? 2 : (t + e < lower ? 0 : 1);
         nin += cl[q] == 2 ? 1 : 0;
-        if (cl[q] == 1) band[atomicAdd(&uscratch[44], 1u)] = ibase + q;
+        if (cl[q] == 1) {
+          const uint32_t m = atomicAdd(&uscratch[44], 1u);
+          band[m] = ibase + q;
+          band_key[m] = 0u;
+        }
       }
     }
 #pragma unroll
@@ -603,8 +609,6 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     __syncthreads();
     const int nband = static_cast<int>(uscratch[44]);
     const int need = n0 - static_cast<int>(uscratch[45]);
-    for (int m = tid; m < nband; m += kThreads) band_key[m] = 0u;
-    __syncthreads();
 
     if constexpr (NC < 4) {
       // ---- canonical fp32 scores of the band: every row of every key
@@ -766,12 +770,28 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     // ---- keep and split: the kept candidates, in start order, become the
     // next round's chunks; their halves (or themselves, when one block long)
     // are written straight into the other candidate buffer
+    int csv[PER], cev[PER];
+    uint8_t kb[PER];
+#pragma unroll
+    for (int v = 0; v < PER / 4; ++v) {
+      int4 x0 = make_int4(0, 0, 0, 0), x1 = x0;
+      uint32_t kw = 0u;
+      if (ibase + 4 * v < ncand) {
+        x0 = reinterpret_cast<const int4*>(cs + ibase)[v];
+        x1 = reinterpret_cast<const int4*>(ce + ibase)[v];
+        kw = reinterpret_cast<const uint32_t*>(keepb + ibase)[v];
+      }
+      csv[4 * v] = x0.x; csv[4 * v + 1] = x0.y; csv[4 * v + 2] = x0.z; csv[4 * v + 3] = x0.w;
+      cev[4 * v] = x1.x; cev[4 * v + 1] = x1.y; cev[4 * v + 2] = x1.z; cev[4 * v + 3] = x1.w;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) kb[4 * v + q] = static_cast<uint8_t>((kw >> (8 * q)) & 0xffu);
+    }
     int cnt = 0, nl = 0;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int i = ibase + q;
-      if (i < ncand && (cl[q] == 2 || (cl[q] == 1 && keepb[i]))) {
-        const int len = ce[i] - cs[i];
+      if (i < ncand && (cl[q] == 2 || (cl[q] == 1 && kb[q]))) {
+        const int len = cev[q] - csv[q];
         cnt += len > 1 ? 2 : 1;
         nl += len > 1 ? 1 : 0;
       } else {
@@ -785,9 +805,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     int* ne = ce_all + (cur ^ 1) * nbuf;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
-      const int i = ibase + q;
       if (cl[q] == 2) {
-        const int s0 = cs[i], e0 = ce[i];
+        const int s0 = csv[q], e0 = cev[q];
         if (e0 - s0 > 1) {
           const int m = s0 + (e0 - s0) / 2;
           ns[pos] = s0; ne[pos] = m; ++pos;
