@@ -529,6 +529,8 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     step_tf = (mask_flops + attn_flops) / (total_ms * 1e-3 / steps) / 1e12
     # hip_mask + hip_sparse_attn (their split merge is fused), or one launch
     launches_per_step = 1 if one_launch else 2
+    if w.dtype == "bf16" and w.group * min(w.block_q, w.q_len) > 32:
+        launches_per_step += 1  # the key-block norm pre-pass of a many-row mask
     two_call = None
     if fused:
         # the same step as the two separate calls, for comparison (not timed above)

@@ -67,6 +67,7 @@ struct MaskPlan {
   int smem;
   size_t ws;
   bool mma;  // tensor-core kernel (bf16) or CUDA-core kernel
+  bool norms;  // key-block norm pre-pass into the workspace (many-row masks)
 };
 
 // Tensor-core mask plan: bf16, up to 256 query rows per mask, b_k <= 32.
@@ -94,6 +95,15 @@ int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
   plan->mma = true;
   plan->ws = kStatusBytes;
+  plan->norms = false;
+  if (nc >= 4) {
+    // many query rows per mask (prefill): the scoring kernel reads the key
+    // norms that bound its tensor-core rounding from a pre-pass over K
+    a.knorm_stride = cdiv(p->seq_len, p->block_k);
+    const size_t bytes = static_cast<size_t>(p->batch) * p->n_kvheads * a.knorm_stride * sizeof(float);
+    plan->ws = kStatusBytes + (bytes + 255) / 256 * 256;
+    plan->norms = true;
+  }
   return HIPS_OK;
 }
 
@@ -118,6 +128,7 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   a.row_stride = row_stride(p);
   a.rows_max = group_rows(p, p->block_q);
   plan->mma = false;
+  plan->norms = false;
   if (plan_mask_mma(p, cluster_cap, plan) == HIPS_OK) return HIPS_OK;
   if (a.rows_max > 32 || a.units > 65535) return HIPS_ERR_UNSUPPORTED;
   const int rc = hips::mask_fma_rc(a.rows_max);
@@ -314,6 +325,11 @@ int launch_mask(const void* q, const void* k, const hips_params* params, int32_t
     hips::MaskArgs& a = plan.a;
     a.q = q; a.k = k; a.idx = idx_out;
     a.status = static_cast<hips::Status*>(params->workspace);
+    if (plan.norms) {
+      a.knorm = reinterpret_cast<const float*>(static_cast<unsigned char*>(params->workspace) + kStatusBytes);
+      const cudaError_t e = hips::launch_key_block_norms(a, params->batch, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
     if (out) {
       if (!fusable(plan)) return HIPS_ERR_UNSUPPORTED;
       a.v = v;

@@ -23,6 +23,10 @@ struct MaskArgs {
   const void* v;
   void* out;
   float scale_log2;
+  // many-row masks: per (sequence, KV head, key block) an upper bound of the
+  // block's key 2-norms, written by key_block_norms before the mask launch
+  const float* knorm;
+  int64_t knorm_stride;  // key blocks per head (ceil(seq_len / block_k))
 };
 
 struct AttnArgs {
@@ -55,6 +59,8 @@ int mask_mma_tile_keys();
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream);
 int mask_mma_fused_rows();  // most query rows of a fused mask + attention launch
+// Fill a.knorm (a workspace array of units' heads x knorm_stride floats)
+cudaError_t launch_key_block_norms(const MaskArgs& a, int batch, cudaStream_t stream);
 
 // Tensor-core attention for query blocks, bf16 (attn_mma.cu)
 int attn_mma_smem_bytes(int table_items);

@@ -166,14 +166,19 @@ __device__ __forceinline__ float tile_row_norm2(const unsigned char* tile, int k
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-// Max of 16 values as a tree (depth 4).
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Max of 16 values as a tree of three-input maxima (8 instructions).
 __device__ __forceinline__ float max16(const float (&v)[16]) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = fmaxf(v[i], v[i + 8]);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
-  return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
+  const float m0 = max3f(v[0], v[1], v[2]), m1 = max3f(v[3], v[4], v[5]);
+  const float m2 = max3f(v[6], v[7], v[8]), m3 = max3f(v[9], v[10], v[11]);
+  const float m4 = max3f(v[12], v[13], v[14]);
+  return fmaxf(max3f(m0, m1, m2), max3f(m3, m4, v[15]));
 }
 
 // Largest accumulator column of this thread's TMEM lane over the operand rows
@@ -377,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   float q2max = 0.0f;
   for (int r = 0; r < N; ++r) q2max = fmaxf(q2max, qn[r]);
   const float eps_scale = kGamma * q2max;  // times |k|_2 (rounded up)
+  const int64_t knorm_base = (static_cast<int64_t>(b) * a.n_kvheads + g) * a.knorm_stride;
   const uint32_t idesc = idesc_bf16_f32(kM, N);
   const int cpt = kM >> lbk;  // candidates per tile
   int gt = 0;                 // tiles of earlier rounds (pipeline position)
@@ -442,9 +448,15 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
           j = rep_key(cf + lc) + (kk & (bk - 1));
           kvalid = j < Tc;
         }
-        if (!timed_out && !mbar_wait(&full[slot], (gi / S) & 1)) timed_out = true;
-        // |k|_2 while the MMA runs
-        const float kn2 = kvalid ? tile_row_norm2(ring + slot * kTileBytes, kk) : 0.0f;
+        // |k|_2 (rounded up) while the MMA runs: the block bound of the
+        // pre-pass when there is one, else from the gathered row
+        float kn = 0.0f;
+        if (a.knorm != nullptr) {
+          if (kvalid) kn = a.knorm[knorm_base + (j >> lbk)];
+        } else {
+          if (!timed_out && !mbar_wait(&full[slot], (gi / S) & 1)) timed_out = true;
+          if (kvalid) kn = sqrtf(tile_row_norm2(ring + slot * kTileBytes, kk)) * kNormUp;
+        }
         if (!timed_out && !mbar_wait(&mma_done[tb], (gi >> 1) & 1)) timed_out = true;
         tc_fence_after_sync();
         __syncwarp();
@@ -479,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
           mbar_arrive(&empty[slot]);
           mbar_arrive(&tm_empty[tb]);
         }
-        float eps = kvalid ? eps_scale * (sqrtf(kn2) * kNormUp) : 0.0f;
+        float eps = kvalid ? eps_scale * kn : 0.0f;
         if (!kvalid) tsc = -INFINITY;
         for (int o = 1; o < bk; o <<= 1) {
           tsc = fmaxf(tsc, __shfl_xor_sync(0xffffffffu, tsc, o));
@@ -1098,6 +1110,42 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   if (C > 1) cluster.sync();  // peers may still read this CTA's scores
 }
 
+// Upper bounds of the key 2-norms per key block: out[head * nblk + blk] =
+// max over the block's keys j < seq_len of |k_j|_2, rounded up. Eight lanes
+// per block (32 bytes of each key row per lane).
+__global__ void __launch_bounds__(kThreads) key_block_norms_kernel(const unsigned char* k, float* out,
+                                                                   int64_t heads, int64_t nblk,
+                                                                   int64_t kv_cap, int64_t seq_len,
+                                                                   int bk) {
+  const int lane8 = threadIdx.x & 7;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * (kThreads / 8) + (threadIdx.x >> 3);
+  if (gid >= heads * nblk) return;  // the whole 8-lane group leaves together
+  const unsigned gmask = 0xffu << (threadIdx.x & 24);
+  const int64_t head = gid / nblk, blk = gid - head * nblk;
+  const unsigned char* base = k + head * kv_cap * 256;
+  float m = 0.0f;
+  for (int kt = 0; kt < bk; ++kt) {
+    const int64_t j = blk * bk + kt;
+    if (j >= seq_len) break;
+    const uint4 x0 = *reinterpret_cast<const uint4*>(base + j * 256 + lane8 * 32);
+    const uint4 x1 = *reinterpret_cast<const uint4*>(base + j * 256 + lane8 * 32 + 16);
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float lo = bf16lo(w[i]), hi = bf16hi(w[i]);
+      s0 = fmaf(lo, lo, s0);
+      s1 = fmaf(hi, hi, s1);
+    }
+    float s = s0 + s1;
+    s += __shfl_xor_sync(gmask, s, 4);
+    s += __shfl_xor_sync(gmask, s, 2);
+    s += __shfl_xor_sync(gmask, s, 1);
+    m = fmaxf(m, s);
+  }
+  if (lane8 == 0) out[gid] = sqrtf(m) * kNormUp;
+}
+
 template <int NC, int PER>
 cudaError_t prepare(const MaskArgs& a, int smem) {
   static int smem_set[kMaxDevices] = {};
@@ -1176,6 +1224,17 @@ int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster) {
 int mask_mma_tile_keys() { return kM; }
 
 int mask_mma_fused_rows() { return 4; }
+
+cudaError_t launch_key_block_norms(const MaskArgs& a, int batch, cudaStream_t stream) {
+  const int64_t heads = static_cast<int64_t>(batch) * a.n_kvheads;
+  const int64_t groups = heads * a.knorm_stride;
+  const int64_t ctas = (groups + kThreads / 8 - 1) / (kThreads / 8);
+  if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+  key_block_norms_kernel<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(
+      static_cast<const unsigned char*>(a.k), const_cast<float*>(a.knorm), heads, a.knorm_stride,
+      a.kv_cap, a.seq_len, a.block_k);
+  return cudaGetLastError();
+}
 
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem) {
   switch (mask_mma_nc(a.rows_max)) {
