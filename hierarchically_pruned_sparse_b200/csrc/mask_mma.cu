@@ -146,6 +146,42 @@ __device__ __forceinline__ void load_row16_sw(const unsigned char* base, int row
   x[12] = bf16lo(b.z); x[13] = bf16hi(b.z); x[14] = bf16lo(b.w); x[15] = bf16hi(b.w);
 }
 
+// Marks of the rows that see key j (as in tmem_row_max) whose accumulator
+// column is >= thr: bit r % 32 of words[r / 32]. Warp-collective.
+template <int NC>
+__device__ __forceinline__ void tmem_row_marks(uint32_t taddr, int R, bool all_rows, int64_t jrel,
+                                               const int* rpos, float thr, uint32_t* words) {
+  constexpr int kBatch = NC < 4 ? NC : 4;
+  static_assert(kBatch % 2 == 0 || NC == 1, "chunk pairs");
+#pragma unroll 1
+  for (int ch0 = 0; ch0 < NC; ch0 += kBatch) {
+    float v[kBatch][16];
+#pragma unroll
+    for (int c = 0; c < kBatch; ++c) tc_ld16(taddr + (ch0 + c) * 16, v[c]);
+    tc_wait_ld();
+    uint32_t bits[kBatch];
+#pragma unroll
+    for (int c = 0; c < kBatch; ++c) {
+      const int r0 = (ch0 + c) * 16;
+      uint32_t b = 0u;
+      if (all_rows && r0 + 16 <= R) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) b |= v[c][i] >= thr ? (1u << i) : 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const bool ok = r0 + i < R && (all_rows || rpos[r0 + i] >= jrel);
+          b |= (ok && v[c][i] >= thr) ? (1u << i) : 0u;
+        }
+      }
+      bits[c] = b;
+    }
+#pragma unroll
+    for (int c = 0; c + 1 < kBatch; c += 2) words[(ch0 + c) >> 1] = bits[c] | (bits[c + 1] << 16);
+    if (kBatch == 1) words[0] = bits[0];
+  }
+}
+
 // Squared 2-norm of key row kk of a swizzled tile.
 __device__ __forceinline__ float tile_row_norm2(const unsigned char* tile, int kk) {
   float acc[8];
@@ -703,26 +739,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
           const float tmax = tmem_row_max<NC>(taddr, R, all_rows, jrel, rpos);  // every lane
           float tstar = kvalid ? tmax - ek : -INFINITY;
           for (int o = 1; o < bk; o <<= 1) tstar = fmaxf(tstar, __shfl_xor_sync(0xffffffffu, tstar, o));
-          const float thr = tstar - ek;
-          uint32_t mw[MW];
-#pragma unroll
-          for (int w = 0; w < MW; ++w) mw[w] = 0u;
-#pragma unroll
-          for (int ch = 0; ch < NC; ++ch) {
-            float v[16];
-            tc_ld16(taddr + ch * 16, v);
-            tc_wait_ld();
-            uint32_t bits = 0u;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int r = ch * 16 + i;
-              const bool ok = kvalid && r < R && (all_rows || rpos[r] >= jrel);
-              bits |= (ok && v[i] >= thr) ? (1u << i) : 0u;
-            }
-            mw[ch >> 1] |= bits << ((ch & 1) * 16);
-          }
-#pragma unroll
-          for (int w = 0; w < MW; ++w) rowmask[kk * MW + w] = mw[w];
+          const float thr = kvalid ? tstar - ek : INFINITY;  // no row of an invalid key
+          tmem_row_marks<NC>(taddr, R, all_rows, jrel, rpos, thr, rowmask + kk * MW);
           tc_fence_before_sync();
         }
         __syncthreads();
