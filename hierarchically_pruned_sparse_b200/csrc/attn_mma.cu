@@ -8,22 +8,25 @@
 // (Author Rebuttal to the Reviewer NLBm, W2: per-row non-zero block indices
 // and nnz).
 //
-// Design: one CTA per (128 query rows of a query block, KV head, sequence);
+// Design: one CTA per (256 query rows of a query block, KV head, sequence);
 // the rows are the group's query heads x positions, so all of them share
-// every gathered K/V tile. Warp roles:
-//  * warps 4-7 gather the keys of the next tiles (64 keys: K and V rows of
-//    the listed blocks) with cp.async into a 3-stage ring, in the tensor-core
+// every gathered K/V tile. They form two M = 128 halves with their own TMEM
+// accumulators (S: 2 x 2 buffers of 64 columns, O: 2 x 128 columns, all 512
+// columns of the SM). Warp roles:
+//  * warps 8-10 gather the keys of the next tiles (64 keys: K and V rows of
+//    the listed blocks) with cp.async into a 2-stage ring, in the tensor-core
 //    layout (K-major, 128-byte swizzle);
-//  * warp 8 issues the MMAs: S = Q K^T (M = 128 rows, N = 64 keys, K = 128)
-//    into one of two TMEM buffers, then O += P V (M = 128, N = 128, K = 64,
-//    V read as an MN-major operand) into the TMEM accumulator; S of tile j+1
-//    is issued before P V of tile j, so the tensor core works while the
-//    softmax of tile j runs;
-//  * warps 0-3 own one query row per thread: read the row of S from TMEM,
-//    mask (causal, invalid slots), keep a reference max and the row sum,
-//    write P (bf16) to shared memory. The reference max only moves (and O
-//    and the sum are rescaled, through TMEM) when a tile's max exceeds it by
-//    more than 2^8, so P stays <= 256 and the result is the exact softmax.
+//  * warp 11 issues the MMAs: S = Q K^T (M = 128 rows, N = 64 keys, K = 128)
+//    for each half into one of two TMEM buffers, then O += P V (M = 128,
+//    N = 128, K = 64, V read as an MN-major operand); S of tile j+1 is issued
+//    before P V of tile j, so the tensor core works while the softmax of
+//    tile j runs;
+//  * warps 0-7 own one query row per thread (warps 0-3 the first half, 4-7
+//    the second): read the row of S from TMEM, mask (causal, invalid slots),
+//    keep a reference max and the row sum, write P (bf16) to shared memory.
+//    The reference max only moves (and O and the sum are rescaled, through
+//    TMEM) when a tile's max exceeds it by more than 2^8, so P stays <= 256
+//    and the result is the exact softmax.
 // All waits are bounded; a timeout sets the status word.
 #include "hips_common.cuh"
 #include "hips_kernels.h"
@@ -33,11 +36,19 @@ namespace hips {
 
 namespace {
 
-constexpr int kRows = 128;                 // query rows per CTA (M)
+constexpr int kRows = 128;                 // query rows per MMA (M)
+constexpr int kHalves = 2;                 // MMA row halves per CTA
+constexpr int kCtaRows = kRows * kHalves;  // query rows per CTA
 constexpr int kKeys = 64;                  // keys per tile
-constexpr int kStages = 3;
-constexpr int kAttnThreads = 288;          // 4 softmax + 4 loader + 1 MMA warps
-constexpr int kQBytes = kRows * 256;       // 32 KB: two 16 KB halves
+constexpr int kStages = 2;
+constexpr int kSoftmax = kCtaRows;         // softmax threads (warps 0-7)
+constexpr int kLoaderWarp0 = kSoftmax / 32;
+constexpr int kLoaders = 96;               // warps 8-10
+constexpr int kMmaWarp = kLoaderWarp0 + kLoaders / 32;
+// 8 softmax + 3 loader + 1 MMA warps: 3 warps per SM sub-partition, so that
+// each thread may hold up to 168 registers
+constexpr int kAttnThreads = (kMmaWarp + 1) * 32;
+constexpr int kQBytes = kRows * 256;       // 32 KB per half: two 16 KB column halves
 constexpr int kKVHalf = kKeys * 128;       // 8 KB
 constexpr int kKVBytes = kKeys * 256;      // 16 KB per K (or V) tile
 constexpr int kPBytes = kRows * 128;       // 16 KB: one row of 64 keys per query row
@@ -52,10 +63,10 @@ __host__ __device__ inline int al2(int x, int a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline AttnMmaSmem attn_mma_layout(int table_items) {
   AttnMmaSmem L;
   int o = 0;
-  L.q = o;     o += kQBytes;
+  L.q = o;     o += kHalves * kQBytes;
   L.k = o;     o += kStages * kKVBytes;
   L.v = o;     o += kStages * kKVBytes;
-  L.p = o;     o += 2 * kPBytes;
+  L.p = o;     o += kHalves * 2 * kPBytes;
   L.bars = o;  o += 16 * 8;
   L.kpos = o;  o += 2 * kKeys * 4;
   L.slot = o;  o += 16;
@@ -71,7 +82,6 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int mt = blockIdx.x;
   const int qb = blockIdx.y % a.nqb, g = blockIdx.y / a.nqb, b = blockIdx.z;
   const int i0 = qb * a.block_q;
   const int nrows = min(a.block_q, a.q_len - i0);
@@ -81,7 +91,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   const int IK = a.item_keys;  // a power of two
   const int lik = __ffs(IK) - 1;
   const int ipt = kKeys >> lik;
-  const int row0 = mt * kRows;
+  const int row0 = blockIdx.x * kCtaRows;
+  const int halves = min(kHalves, (R - row0 + kRows - 1) / kRows);  // halves with rows (>= 1)
 
   const AttnMmaSmem L = attn_mma_layout(a.table_items);
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -90,10 +101,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   unsigned char* vs = smem + L.v;
   unsigned char* ps = smem + L.p;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* kv_full = bars;        // [3] cp.async arrivals of the 128 loader threads
-  uint64_t* kv_empty = bars + 3;   // [3] P V of the tile in the stage done
-  uint64_t* s_full = bars + 6;     // [2] S MMA done
-  uint64_t* p_full = bars + 8;     // [2] P written by the 128 softmax threads
+  uint64_t* kv_full = bars;        // [kStages] cp.async arrivals of the loader threads
+  uint64_t* kv_empty = bars + 3;   // [kStages] P V of the tile in the stage done
+  uint64_t* s_full = bars + 6;     // [2] S MMAs (both halves) done
+  uint64_t* p_full = bars + 8;     // [2] P written by the softmax threads
   uint64_t* pv_done = bars + 10;   // [2] P V MMA done
   int* kpos = reinterpret_cast<int*>(smem + L.kpos);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L.slot);
@@ -101,30 +112,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 128);
+      mbar_init(&kv_full[s], kLoaders);
       mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], kSoftmax);
       mbar_init(&pv_done[s], 1);
     }
     fence_mbar_init();
   }
   __syncwarp();
-  if (warp == 0) tmem_alloc(tslot, 256);
-  // query rows of this CTA in the operand layout (rows >= R are zero)
+  if (warp == 0) tmem_alloc(tslot, 512);
+  // query rows of this CTA in the operand layout, one 128-row half after the
+  // other (rows >= R are zero)
   const uint16_t* qg = static_cast<const uint16_t*>(a.q);
-  for (int i = tid; i < kRows * 16; i += kAttnThreads) {
-    const int r = i >> 4, c = i & 15;
-    const int ur = row0 + r;
+  for (int i = tid; i < kCtaRows * 16; i += kAttnThreads) {
+    const int rq = i >> 4, c = i & 15;
+    const int ur = row0 + rq, r = rq & (kRows - 1);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (ur < R) {
       const int h = g * a.group + ur / nrows, qi = i0 + ur % nrows;
       v = *reinterpret_cast<const uint4*>(
           qg + ((static_cast<int64_t>(b) * a.n_qheads + h) * a.q_len + qi) * kD + c * 8);
     }
-    *reinterpret_cast<uint4*>(qs + (c >> 3) * (kQBytes / 2) + sw128_offset(r, c & 7)) = v;
+    *reinterpret_cast<uint4*>(qs + (rq >> 7) * kQBytes + (c >> 3) * (kQBytes / 2) +
+                              sw128_offset(r, c & 7)) = v;
   }
   // the idx rows may come from the kernel launched just before this one
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -164,24 +177,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tslot;
-  const uint32_t tmem_o = tmem + 128;
+  const uint32_t tmem_o = tmem + 256;  // O of half h at columns 256 + 128 h
   bool timed_out = false;
 
   const size_t plane = (static_cast<size_t>(b) * a.n_kvheads + g) * static_cast<size_t>(a.kv_cap) * 256;
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) + plane;
   const unsigned char* vbase = static_cast<const unsigned char*>(a.v) + plane;
 
-  if (warp >= 4 && warp < 8) {
-    // ---------------- loaders: K and V rows of tile j into stage j % 3
-    const int lt = tid - 128;
+  if (warp >= kLoaderWarp0 && warp < kMmaWarp) {
+    // ---------------- loaders: K and V rows of tile j into stage j % kStages
+    const int lt = tid - kSoftmax;
     for (int j = 0; j < ntiles; ++j) {
       const int st = j % kStages;
       if (j >= kStages && !mbar_wait(&kv_empty[st], ((j - kStages) / kStages) & 1)) timed_out = true;
       unsigned char* kd = ks + st * kKVBytes;
       unsigned char* vd = vs + st * kKVBytes;
-#pragma unroll
-      for (int m = 0; m < (kKeys * 16) / 128; ++m) {
-        const int i = lt + 128 * m;
+#pragma unroll 4
+      for (int i = lt; i < kKeys * 16; i += kLoaders) {
         const int kk = i >> 4, ch = i & 15;
         const int item = j * ipt + (kk >> lik), kt = kk & (IK - 1);
         if (item < nitems) {
@@ -196,7 +208,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
       }
       cp_async_arrive(&kv_full[st]);
     }
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issue (one thread)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kRows, kKeys);
@@ -205,11 +217,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         const int psb = pj & 1, pst = pj % kStages;
         if (!mbar_wait(&p_full[psb], (pj >> 1) & 1)) timed_out = true;
         tc_fence_after_sync();
+        for (int h = 0; h < halves; ++h) {
 #pragma unroll
-        for (int k = 0; k < kKeys / 16; ++k) {
-          const uint64_t ad = sw128_desc(smem_u32(ps + psb * kPBytes) + k * 32);
-          const uint64_t bd = sw128_desc_mn(smem_u32(vs + pst * kKVBytes) + k * 2048, kKVHalf);
-          tc_mma_bf16(tmem_o, ad, bd, idesc_o, (pj > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < kKeys / 16; ++k) {
+            const uint64_t ad = sw128_desc(smem_u32(ps + (h * 2 + psb) * kPBytes) + k * 32);
+            const uint64_t bd = sw128_desc_mn(smem_u32(vs + pst * kKVBytes) + k * 2048, kKVHalf);
+            tc_mma_bf16(tmem_o + h * 128, ad, bd, idesc_o, (pj > 0 || k > 0) ? 1u : 0u);
+          }
         }
         tc_commit(&pv_done[psb]);
         tc_commit(&kv_empty[pst]);
@@ -218,11 +232,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         const int st = j % kStages, sb = j & 1;
         if (!mbar_wait(&kv_full[st], (j / kStages) & 1)) timed_out = true;
         tc_fence_after_sync();
+        for (int h = 0; h < halves; ++h) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t ad = sw128_desc(smem_u32(qs + (k >> 2) * (kQBytes / 2)) + (k & 3) * 32);
-          const uint64_t bd = sw128_desc(smem_u32(ks + st * kKVBytes + (k >> 2) * kKVHalf) + (k & 3) * 32);
-          tc_mma_bf16(tmem + sb * kKeys, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t ad =
+                sw128_desc(smem_u32(qs + h * kQBytes + (k >> 2) * (kQBytes / 2)) + (k & 3) * 32);
+            const uint64_t bd = sw128_desc(smem_u32(ks + st * kKVBytes + (k >> 2) * kKVHalf) + (k & 3) * 32);
+            tc_mma_bf16(tmem + h * 128 + sb * kKeys, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          }
         }
         tc_commit(&s_full[sb]);
         if (j >= 1) issue_pv(j - 1);
@@ -231,11 +248,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
     }
     __syncwarp();
   } else {
-    // ---------------- softmax: thread tid owns query row row0 + tid
+    // ---------------- softmax: thread tid owns query row row0 + tid, of
+    // half h = tid / 128 (TMEM lane tid % 128)
+    const int hh = tid >> 7, rr = tid & (kRows - 1);
+    const uint32_t s_col = tmem + hh * 128;   // S buffers of this half
+    const uint32_t o_col = tmem_o + hh * 128;  // O of this half
     const int ur = row0 + tid;
     const bool row_ok = ur < R;
     const int64_t my_pos = q_first + (row_ok ? ur % nrows : 0);
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lane quarter
     float m_ref = -INFINITY, lsum = 0.0f;
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
@@ -248,7 +269,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         }
         kpos[sb * kKeys + tid] = kp;
       }
-      named_sync(1, 128);
+      named_sync(1, kSoftmax);
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1)) timed_out = true;
       tc_fence_after_sync();
       __syncwarp();
@@ -256,7 +277,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
 #pragma unroll
       for (int c = 0; c < kKeys / 16; ++c) {
         float v[16];
-        tc_ld16(tmem + lane_base + sb * kKeys + c * 16, v);
+        tc_ld16(s_col + lane_base + sb * kKeys + c * 16, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) s[c * 16 + i] = v[i];
       }
@@ -284,11 +305,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
 #pragma unroll
         for (int c = 0; c < kD / 16; ++c) {
           float v[16];
-          tc_ld16(tmem_o + lane_base + c * 16, v);
+          tc_ld16(o_col + lane_base + c * 16, v);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] *= alpha;
-          tc_st16(tmem_o + lane_base + c * 16, v);
+          tc_st16(o_col + lane_base + c * 16, v);
         }
         tc_wait_st();
       }
@@ -296,25 +317,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         lsum *= alpha;
         m_ref = tmax;
       }
-      float p[kKeys];
-      float psum = 0.0f;
+      float psum = 0.0f;  // P overwrites S in place
 #pragma unroll
       for (int i = 0; i < kKeys; ++i) {
-        p[i] = s[i] == -INFINITY ? 0.0f : exp2f(s[i] - m_ref);
-        psum += p[i];
+        s[i] = s[i] == -INFINITY ? 0.0f : exp2f(s[i] - m_ref);
+        psum += s[i];
       }
       lsum += psum;
       // P buffer sb is free once P V of tile j - 2 is done
       if (j >= 2 && !mbar_wait(&pv_done[sb], ((j - 2) >> 1) & 1)) timed_out = true;
-      unsigned char* prow = ps + sb * kPBytes;
+      unsigned char* prow = ps + (hh * 2 + sb) * kPBytes;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 w;
-        w.x = pack_bf16x2(p[c * 8 + 0], p[c * 8 + 1]);
-        w.y = pack_bf16x2(p[c * 8 + 2], p[c * 8 + 3]);
-        w.z = pack_bf16x2(p[c * 8 + 4], p[c * 8 + 5]);
-        w.w = pack_bf16x2(p[c * 8 + 6], p[c * 8 + 7]);
-        *reinterpret_cast<uint4*>(prow + sw128_offset(tid, c)) = w;
+        w.x = pack_bf16x2(s[c * 8 + 0], s[c * 8 + 1]);
+        w.y = pack_bf16x2(s[c * 8 + 2], s[c * 8 + 3]);
+        w.z = pack_bf16x2(s[c * 8 + 4], s[c * 8 + 5]);
+        w.w = pack_bf16x2(s[c * 8 + 6], s[c * 8 + 7]);
+        *reinterpret_cast<uint4*>(prow + sw128_offset(rr, c)) = w;
       }
       fence_proxy_async_smem();
       tc_fence_before_sync();
@@ -336,7 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
     for (int c = 0; c < kD / 16; ++c) {
       float v[16];
       if (ntiles > 0) {
-        tc_ld16(tmem_o + lane_base + c * 16, v);
+        tc_ld16(o_col + lane_base + c * 16, v);
         tc_wait_ld();
       } else {
 #pragma unroll
@@ -359,14 +379,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   if (timed_out) report(a.status, kStatusTimeout, 4);
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
 
 int attn_mma_smem_bytes(int table_items) { return attn_mma_layout(table_items).total; }
 int attn_mma_tile_keys() { return kKeys; }
-int attn_mma_rows() { return kRows; }
+int attn_mma_rows() { return kCtaRows; }
 
 cudaError_t launch_attn_mma(const AttnArgs& a, int smem, cudaStream_t stream) {
   static int smem_set[kMaxDevices] = {};
@@ -380,7 +400,7 @@ cudaError_t launch_attn_mma(const AttnArgs& a, int smem, cudaStream_t stream) {
     smem_set[dev] = smem;
   }
   cudaLaunchConfig_t cfg = {};
-  const int mtiles = (a.rows_max + kRows - 1) / kRows;
+  const int mtiles = (a.rows_max + kCtaRows - 1) / kCtaRows;
   cfg.gridDim = dim3(mtiles, a.nqb * a.n_kvheads, a.batch);
   cfg.blockDim = dim3(kAttnThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
