@@ -14,7 +14,7 @@
 // accumulators (S: 2 x 2 buffers of 64 columns, O: 2 x 128 columns, all 512
 // columns of the SM). Warp roles:
 //  * warps 8-10 gather the keys of the next tiles (64 keys: K and V rows of
-//    the listed blocks) with cp.async into a 2-stage ring, in the tensor-core
+//    the listed blocks) with cp.async into a 3-stage ring, in the tensor-core
 //    layout (K-major, 128-byte swizzle);
 //  * warp 11 issues the MMAs: S = Q K^T (M = 128 rows, N = 64 keys, K = 128)
 //    for each half into one of two TMEM buffers, then O += P V (M = 128,
@@ -40,7 +40,7 @@ constexpr int kRows = 128;                 // query rows per MMA (M)
 constexpr int kHalves = 2;                 // MMA row halves per CTA
 constexpr int kCtaRows = kRows * kHalves;  // query rows per CTA
 constexpr int kKeys = 64;                  // keys per tile
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kSoftmax = kCtaRows;         // softmax threads (warps 0-7)
 constexpr int kLoaderWarp0 = kSoftmax / 32;
 constexpr int kLoaders = 96;               // warps 8-10
@@ -66,9 +66,9 @@ __host__ __device__ inline AttnMmaSmem attn_mma_layout(int table_items) {
   L.q = o;     o += kHalves * kQBytes;
   L.k = o;     o += kStages * kKVBytes;
   L.v = o;     o += kStages * kKVBytes;
-  L.p = o;     o += kHalves * 2 * kPBytes;
+  L.p = o;     o += kHalves * kPBytes;  // one P tile per half
   L.bars = o;  o += 16 * 8;
-  L.kpos = o;  o += 2 * kKeys * 4;
+  L.kpos = o;  o += 2 * kKeys * 4 + 16;  // key positions of two tiles, then their flags
   L.slot = o;  o += 16;
   L.table = o; o += al2(table_items * 8, 16);
   L.total = o + 1024;
@@ -192,17 +192,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
       if (j >= kStages && !mbar_wait(&kv_empty[st], ((j - kStages) / kStages) & 1)) timed_out = true;
       unsigned char* kd = ks + st * kKVBytes;
       unsigned char* vd = vs + st * kKVBytes;
-#pragma unroll 4
-      for (int i = lt; i < kKeys * 16; i += kLoaders) {
-        const int kk = i >> 4, ch = i & 15;
+      // two threads per key row (8 of its 16 chunks each, K and V): one
+      // table lookup per row and thread
+      for (int kk = lt >> 1; kk < kKeys; kk += kLoaders / 2) {
         const int item = j * ipt + (kk >> lik), kt = kk & (IK - 1);
         if (item < nitems) {
           const int2 e = table[item];
           if (kt < e.y) {
-            const size_t src = (static_cast<size_t>(e.x) + kt) * 256 + ch * 16;
-            const uint32_t dst = (ch >> 3) * kKVHalf + sw128_offset(kk, ch & 7);
-            cp_async16(kd + dst, kbase + src);
-            cp_async16(vd + dst, vbase + src);
+            const size_t row = (static_cast<size_t>(e.x) + kt) * 256;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int ch = (lt & 1) + 2 * q;
+              const uint32_t dst = (ch >> 3) * kKVHalf + sw128_offset(kk, ch & 7);
+              cp_async16(kd + dst, kbase + row + ch * 16);
+              cp_async16(vd + dst, vbase + row + ch * 16);
+            }
           }
         }
       }
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         for (int h = 0; h < halves; ++h) {
 #pragma unroll
           for (int k = 0; k < kKeys / 16; ++k) {
-            const uint64_t ad = sw128_desc(smem_u32(ps + (h * 2 + psb) * kPBytes) + k * 32);
+            const uint64_t ad = sw128_desc(smem_u32(ps + h * kPBytes) + k * 32);
             const uint64_t bd = sw128_desc_mn(smem_u32(vs + pst * kKVBytes) + k * 2048, kKVHalf);
             tc_mma_bf16(tmem_o + h * 128, ad, bd, idesc_o, (pj > 0 || k > 0) ? 1u : 0u);
           }
@@ -268,8 +272,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
           if (kt < e.y) kp = e.x + kt;
         }
         kpos[sb * kKeys + tid] = kp;
+        // flag: every key of this half-tile is valid and seen by every row
+        const bool seen = __all_sync(0xffffffffu, kp >= 0 && kp <= q_first);
+        if (lane == 0) kpos[2 * kKeys + sb * 2 + warp] = seen ? 1 : 0;
       }
       named_sync(1, kSoftmax);
+      const bool all_seen = kpos[2 * kKeys + sb * 2] && kpos[2 * kKeys + sb * 2 + 1];
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1)) timed_out = true;
       tc_fence_after_sync();
       __syncwarp();
@@ -282,17 +290,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         for (int i = 0; i < 16; ++i) s[c * 16 + i] = v[i];
       }
       tc_wait_ld();
-      float tmax = -INFINITY;
+      float tmax;
+      if (all_seen) {
+        // no masking: the max of the raw scores times the (positive) scale
+        float m[8];
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 4) {
-        const int4 kp4 = *reinterpret_cast<const int4*>(kpos + sb * kKeys + c);
-        const int kp[4] = {kp4.x, kp4.y, kp4.z, kp4.w};
+        for (int i = 0; i < 8; ++i) m[i] = max3f(s[i], s[8 + i], max3f(s[16 + i], s[24 + i], s[32 + i]));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const bool ok = row_ok && kp[i] >= 0 && kp[i] <= my_pos;
-          s[c + i] = ok ? s[c + i] * a.scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, s[c + i]);
+        for (int i = 0; i < 8; ++i) m[i] = max3f(m[i], s[40 + i], max3f(s[48 + i], s[56 + i], m[i]));
+        tmax = max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7])) * a.scale_log2;
+      } else {
+        float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < kKeys; c += 4) {
+          const int4 kp4 = *reinterpret_cast<const int4*>(kpos + sb * kKeys + c);
+          const int kp[4] = {kp4.x, kp4.y, kp4.z, kp4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const bool ok = row_ok && kp[i] >= 0 && kp[i] <= my_pos;
+            s[c + i] = ok ? s[c + i] * a.scale_log2 : -INFINITY;
+            m[i] = fmaxf(m[i], s[c + i]);
+          }
         }
+        tmax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
       }
       // move the reference max only when this tile exceeds it by > 2^8
       const bool grow = tmax > m_ref + kRescaleLog2;
@@ -317,16 +337,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         lsum *= alpha;
         m_ref = tmax;
       }
-      float psum = 0.0f;  // P overwrites S in place
+      // P overwrites S in place; four partial sums
+      float ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (all_seen) {
+        const float nm = -m_ref;
 #pragma unroll
-      for (int i = 0; i < kKeys; ++i) {
-        s[i] = s[i] == -INFINITY ? 0.0f : exp2f(s[i] - m_ref);
-        psum += s[i];
+        for (int i = 0; i < kKeys; ++i) {
+          s[i] = exp2f(fmaf(s[i], a.scale_log2, nm));
+          ps4[i & 3] += s[i];
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kKeys; ++i) {
+          s[i] = s[i] == -INFINITY ? 0.0f : exp2f(s[i] - m_ref);
+          ps4[i & 3] += s[i];
+        }
       }
-      lsum += psum;
+      lsum += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
       // P buffer sb is free once P V of tile j - 2 is done
-      if (j >= 2 && !mbar_wait(&pv_done[sb], ((j - 2) >> 1) & 1)) timed_out = true;
-      unsigned char* prow = ps + (hh * 2 + sb) * kPBytes;
+      // the P tile of this half is free once P V of tile j - 1 is done
+      if (j >= 1 && !mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) timed_out = true;
+      unsigned char* prow = ps + hh * kPBytes;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 w;

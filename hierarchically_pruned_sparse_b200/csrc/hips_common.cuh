@@ -124,6 +124,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Order-preserving map of a float score onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t score_key(float f) {
   if (f == 0.0f) f = 0.0f;  // -0 and +0 are the same score

@@ -202,13 +202,6 @@ __device__ __forceinline__ float tile_row_norm2(const unsigned char* tile, int k
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-// Three-input maximum (one instruction on sm_100).
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Max of 16 values as a tree of three-input maxima (8 instructions).
 __device__ __forceinline__ float max16(const float (&v)[16]) {
   const float m0 = max3f(v[0], v[1], v[2]), m1 = max3f(v[3], v[4], v[5]);
