@@ -64,8 +64,12 @@ constexpr int kProducerWarp0 = 5;       // warps 5-7 gather key tiles
 constexpr int kProducers = (kWarps - kProducerWarp0) * 32;
 
 __host__ __device__ constexpr int stages_for(int nc, int per) {
-  return per > 8 ? 2 : nc >= 16 ? 2 : nc >= 8 ? 3 : 4;
+  return per > 8 ? 2 : nc >= 8 ? 3 : 4;
 }
+// Many-row masks keep the arrays that only the selection uses (histogram,
+// band lists, keep flags, row marks) in the last ring slot, which the
+// selection never needs: that is what makes room for the slot.
+__host__ __device__ constexpr bool select_in_ring(int nc, int per) { return nc >= 4 && per <= 8; }
 __host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 32 < 32 ? 32 : nc * 32; }
 __host__ __device__ constexpr int mask_words(int nc) { return nc < 2 ? 1 : nc / 2; }
 
@@ -93,14 +97,18 @@ __host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cl
   L.qn = o;       o += nc * 16 * 4;  // |q_r|_2, rounded up (0 for padding rows)
   L.cs = o;       o += 2 * n * 4;
   L.ce = o;       o += 2 * n * 4;
-  L.keepb = o;    o += al(n, 16);
-  L.band = o;     o += n * 4;
-  L.band_key = o; o += n * 4;
   L.xch = o;      o += (cluster > 1 ? 2 : 1) * n * 8;
-  L.hist = o;     o += kBuckets * 4;
-  L.rowmask = o;  o += nc >= 4 ? kM * mask_words(nc) * 4 : 0;
+  int sel = o;  // selection-only arrays: here, or in the last ring slot
+  if (select_in_ring(nc, per)) sel = L.ring + (S - 1) * kTileBytes;
+  L.band = sel;     sel += n * 4;
+  L.band_key = sel; sel += n * 4;
+  L.hist = sel;     sel += kBuckets * 4;
+  L.rowmask = sel;  sel += nc >= 4 ? kM * mask_words(nc) * 4 : 0;
+  L.keepb = sel;    sel += al(n, 16);
+  if (!select_in_ring(nc, per)) o = sel;
   L.scratch = o;  o += 64 * 4;
   L.total = o + 1024;  // room to align the base to 1024 bytes
+  if (select_in_ring(nc, per) && sel > L.ring + S * kTileBytes) L.total = 1 << 30;  // does not fit
   return L;
 }
 
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     const int ntiles = (c_hi - c_lo + cpt - 1) / cpt;
     float2* my_x = xch + buf * nbuf;  // indexed by candidate
 
-    if (warp >= kProducerWarp0) {
+    if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducers / 32) {
       // ---------------- gather tiles into the ring
       const int p = tid - kProducerWarp0 * 32;
       for (int t = 0; t < ntiles; ++t) {
@@ -580,6 +588,10 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       uscratch[45] = 0u;           // sure-in count
       uscratch[46] = 0xffffffffu;  // min score key in the cut bucket
       uscratch[47] = 0u;           // max score key in the cut bucket
+    }
+    if constexpr (select_in_ring(NC, PER)) {
+      // the histogram shares a ring slot with this round's tiles
+      for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
     }
     __syncthreads();
     lo = fscratch[16]; hi = fscratch[24]; emax = fscratch[32];
