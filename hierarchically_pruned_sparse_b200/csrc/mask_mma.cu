@@ -74,8 +74,8 @@ __host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 32 < 32 ? 
 __host__ __device__ constexpr int mask_words(int nc) { return nc < 2 ? 1 : nc / 2; }
 
 struct MmaSmem {
-  int ring, bq, bar, slot, rpos, qn, cs, ce, keepb, band, band_key, xch, hist, rowmask, scratch,
-      total;
+  int ring, bq, bar, slot, rpos, qn, cs, ce, keepb, band, band_key, xch, hist, rowmask, vmask,
+      scratch, total;
 };
 
 __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
@@ -106,6 +106,9 @@ __host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cl
   L.rowmask = sel;  sel += nc >= 4 ? kM * mask_words(nc) * 4 : 0;
   L.keepb = sel;    sel += al(n, 16);
   if (!select_in_ring(nc, per)) o = sel;
+  // rows that see a key d positions past the first row of the query block:
+  // words [d * MW, (d + 1) * MW) (many-row masks)
+  L.vmask = o;    o += nc >= 4 ? nc * 16 * mask_words(nc) * 4 : 0;
   L.scratch = o;  o += 64 * 4;
   L.total = o + 1024;  // room to align the base to 1024 bytes
   if (select_in_ring(nc, per) && sel > L.ring + S * kTileBytes) L.total = 1 << 30;  // does not fit
@@ -154,11 +157,11 @@ __device__ __forceinline__ void load_row16_sw(const unsigned char* base, int row
   x[12] = bf16lo(b.z); x[13] = bf16hi(b.z); x[14] = bf16lo(b.w); x[15] = bf16hi(b.w);
 }
 
-// Marks of the rows that see key j (as in tmem_row_max) whose accumulator
+// Marks of the rows that see the key (as in tmem_row_max) whose accumulator
 // column is >= thr: bit r % 32 of words[r / 32]. Warp-collective.
 template <int NC>
-__device__ __forceinline__ void tmem_row_marks(uint32_t taddr, int R, bool all_rows, int64_t jrel,
-                                               const int* rpos, float thr, uint32_t* words) {
+__device__ __forceinline__ void tmem_row_marks(uint32_t taddr, int R, const uint32_t* vrow,
+                                               float thr, uint32_t* words) {
   constexpr int kBatch = NC < 4 ? NC : 4;
   static_assert(kBatch % 2 == 0 || NC == 1, "chunk pairs");
 #pragma unroll 1
@@ -172,13 +175,14 @@ __device__ __forceinline__ void tmem_row_marks(uint32_t taddr, int R, bool all_r
     for (int c = 0; c < kBatch; ++c) {
       const int r0 = (ch0 + c) * 16;
       uint32_t b = 0u;
-      if (all_rows && r0 + 16 <= R) {
+      if (vrow == nullptr && r0 + 16 <= R) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) b |= v[c][i] >= thr ? (1u << i) : 0u;
       } else {
+        const uint32_t w = vrow ? vrow[r0 >> 5] >> (r0 & 31) : 0xffffu;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const bool ok = r0 + i < R && (all_rows || rpos[r0 + i] >= jrel);
+          const bool ok = r0 + i < R && ((w >> i) & 1u);
           b |= (ok && v[c][i] >= thr) ? (1u << i) : 0u;
         }
       }
@@ -219,11 +223,11 @@ __device__ __forceinline__ float max16(const float (&v)[16]) {
 }
 
 // Largest accumulator column of this thread's TMEM lane over the operand rows
-// that see key j: rows [0, R) when every row does (all_rows), else the rows r
-// with rpos[r] >= jrel. Warp-collective (every lane of the warp calls it).
+// that see its key: rows [0, R) when vrow is null (every row does), else the
+// rows whose bit is set in vrow (bit r % 32 of vrow[r / 32]). Warp-collective
+// (every lane of the warp calls it).
 template <int NC>
-__device__ __forceinline__ float tmem_row_max(uint32_t taddr, int R, bool all_rows, int64_t jrel,
-                                              const int* rpos) {
+__device__ __forceinline__ float tmem_row_max(uint32_t taddr, int R, const uint32_t* vrow) {
   constexpr int kBatch = NC < 4 ? NC : 4;
   float acc[kBatch];
 #pragma unroll
@@ -237,13 +241,14 @@ __device__ __forceinline__ float tmem_row_max(uint32_t taddr, int R, bool all_ro
 #pragma unroll
     for (int c = 0; c < kBatch; ++c) {
       const int r0 = (ch0 + c) * 16;
-      if (all_rows && r0 + 16 <= R) {
+      if (vrow == nullptr && r0 + 16 <= R) {
         acc[c] = fmaxf(acc[c], max16(v[c]));
       } else {
+        const uint32_t w = vrow ? vrow[r0 >> 5] >> (r0 & 31) : 0xffffu;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const bool ok = r0 + i < R && (all_rows || rpos[r0 + i] >= jrel);
-          if (ok) acc[c] = fmaxf(acc[c], v[c][i]);
+          const bool ok = r0 + i < R && ((w >> i) & 1u);
+          acc[c] = fmaxf(acc[c], ok ? v[c][i] : -INFINITY);
         }
       }
     }
@@ -326,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   float2* xch = reinterpret_cast<float2*>(smem + L.xch);
   int* hist = reinterpret_cast<int*>(smem + L.hist);
   uint32_t* rowmask = reinterpret_cast<uint32_t*>(smem + L.rowmask);
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + L.vmask);
   int* scratch = reinterpret_cast<int*>(smem + L.scratch);
   float* fscratch = reinterpret_cast<float*>(scratch);
   uint32_t* uscratch = reinterpret_cast<uint32_t*>(scratch);
@@ -363,6 +369,17 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   }
   for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
   for (int r = tid; r < N; r += kThreads) rpos[r] = r < R ? r % nrows : -1;  // -1: padding row
+  if constexpr (NC >= 4) {
+    for (int i = tid; i < N * MW; i += kThreads) {
+      const int d = i / MW, w = i - d * MW;
+      uint32_t bits = 0u;
+      for (int bb = 0; bb < 32; ++bb) {
+        const int r = w * 32 + bb;
+        if (r < R && r % nrows >= d) bits |= 1u << bb;
+      }
+      vmask[i] = bits;
+    }
+  }
   // |q_r|_2 of every row (one warp per row), rounded up
   for (int r = warp; r < N; r += kWarps) {
     float s = 0.0f;
@@ -500,8 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         // every row sees key j when j <= q_first; else row r needs r % b_q >= j - q_first
         float tsc = -INFINITY;
         if constexpr (NC >= 4) {
-          tsc = tmem_row_max<NC>(tmem + (static_cast<uint32_t>(warp * 32) << 16) + tb * N, R,
-                                 j <= q_first, j - q_first, rpos);
+          const uint32_t* vrow =
+              j <= q_first ? nullptr : vmask + static_cast<int>(min64(j - q_first, N - 1)) * MW;
+          tsc = tmem_row_max<NC>(tmem + (static_cast<uint32_t>(warp * 32) << 16) + tb * N, R, vrow);
         } else {
           const bool all_rows = j <= q_first;
           const int64_t jrel = j - q_first;
@@ -736,16 +754,16 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
           if (!timed_out && !mbar_wait(band_bar, band_phase)) timed_out = true;
           tc_fence_after_sync();
           __syncwarp();
-          const bool all_rows = j <= q_first;
-          const int64_t jrel = j - q_first;
+          const uint32_t* vrow =
+              !kvalid || j <= q_first ? nullptr : vmask + static_cast<int>(min64(j - q_first, N - 1)) * MW;
           const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
           // s >= max over the candidate's keys of (t_max - eps): rows below
           // that by more than their key's eps cannot hold the maximum
-          const float tmax = tmem_row_max<NC>(taddr, R, all_rows, jrel, rpos);  // every lane
+          const float tmax = tmem_row_max<NC>(taddr, R, vrow);  // every lane
           float tstar = kvalid ? tmax - ek : -INFINITY;
           for (int o = 1; o < bk; o <<= 1) tstar = fmaxf(tstar, __shfl_xor_sync(0xffffffffu, tstar, o));
           const float thr = kvalid ? tstar - ek : INFINITY;  // no row of an invalid key
-          tmem_row_marks<NC>(taddr, R, all_rows, jrel, rpos, thr, rowmask + kk * MW);
+          tmem_row_marks<NC>(taddr, R, vrow, thr, rowmask + kk * MW);
           tc_fence_before_sync();
         }
         __syncthreads();
