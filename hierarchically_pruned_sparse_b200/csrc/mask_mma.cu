@@ -370,14 +370,18 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
   for (int r = tid; r < N; r += kThreads) rpos[r] = r < R ? r % nrows : -1;  // -1: padding row
   if constexpr (NC >= 4) {
-    for (int i = tid; i < N * MW; i += kThreads) {
-      const int d = i / MW, w = i - d * MW;
-      uint32_t bits = 0u;
-      for (int bb = 0; bb < 32; ++bb) {
-        const int r = w * 32 + bb;
-        if (r < R && r % nrows >= d) bits |= 1u << bb;
+    // thread d fills row d of the table; rm runs through r % b_q
+    for (int d = tid; d < N; d += kThreads) {
+      int rm = 0;
+      for (int w = 0; w < MW; ++w) {
+        uint32_t bits = 0u;
+        for (int bb = 0; bb < 32; ++bb) {
+          const int r = w * 32 + bb;
+          if (r < R && rm >= d) bits |= 1u << bb;
+          rm = rm + 1 == nrows ? 0 : rm + 1;
+        }
+        vmask[d * MW + w] = bits;
       }
-      vmask[i] = bits;
     }
   }
   // |q_r|_2 of every row (one warp per row), rounded up
@@ -492,21 +496,35 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     } else {
       // ---------------- read back: thread = key kk of the tile
       const int kk = warp * 32 + lane;
+      const int lc = kk >> lbk;
+      // key of this thread in tile t (-1 if none)
+      auto key_in_tile = [&](int t) -> int64_t {
+        const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
+        if (lc >= cc) return -1;
+        const int64_t jj = rep_key(cf + lc) + (kk & (bk - 1));
+        return jj < Tc ? jj : -1;
+      };
+      // the pre-pass's block bound of |k|_2 is fetched one tile ahead
+      float kn_next = 0.0f;
+      if (a.knorm != nullptr && ntiles > 0) {
+        const int64_t j0 = key_in_tile(0);
+        if (j0 >= 0) kn_next = a.knorm[knorm_base + (j0 >> lbk)];
+      }
       for (int t = 0; t < ntiles; ++t) {
         const int gi = gt + t, slot = gi % S, tb = gi & 1;
         const int cf = c_lo + t * cpt, cc = min(cpt, c_hi - cf);
-        const int lc = kk >> lbk;
-        bool kvalid = lc < cc;
-        int64_t j = 0;
-        if (kvalid) {
-          j = rep_key(cf + lc) + (kk & (bk - 1));
-          kvalid = j < Tc;
-        }
+        const int64_t jk = key_in_tile(t);
+        const bool kvalid = jk >= 0;
+        const int64_t j = kvalid ? jk : 0;
         // |k|_2 (rounded up) while the MMA runs: the block bound of the
         // pre-pass when there is one, else from the gathered row
         float kn = 0.0f;
         if (a.knorm != nullptr) {
-          if (kvalid) kn = a.knorm[knorm_base + (j >> lbk)];
+          kn = kn_next;
+          if (t + 1 < ntiles) {
+            const int64_t j1 = key_in_tile(t + 1);
+            kn_next = j1 >= 0 ? a.knorm[knorm_base + (j1 >> lbk)] : 0.0f;
+          }
         } else {
           if (!timed_out && !mbar_wait(&full[slot], (gi / S) & 1)) timed_out = true;
           if (kvalid) kn = sqrtf(tile_row_norm2(ring + slot * kTileBytes, kk)) * kNormUp;
