@@ -44,7 +44,7 @@ class Shape(ctypes.Structure):
         ("pad0", ctypes.c_int32), ("q_pos0", ctypes.c_int64),
         ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("topk", ctypes.c_int32), ("sink", ctypes.c_int32),
-        ("window", ctypes.c_int32), ("pad1", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("per_head", ctypes.c_int32),
     ]
 
 
@@ -89,12 +89,14 @@ def _f32(a) -> np.ndarray:
 
 
 def shape(*, batch, n_qheads, n_kvheads, head_dim, seq_len, q_len, q_pos0, block_q,
-          block_k, topk, sink=0, window=0, mask_len=None, kv_capacity=None) -> Shape:
+          block_k, topk, sink=0, window=0, mask_len=None, kv_capacity=None, per_head=0) -> Shape:
+    """per_head=1: one mask per query head (idx rows [B, Hq, n_qblocks]) instead of
+    one per KV-head group."""
     return Shape(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, head_dim=head_dim,
                  seq_len=seq_len, mask_len=seq_len if mask_len is None else mask_len,
                  kv_capacity=seq_len if kv_capacity is None else kv_capacity,
                  q_len=q_len, pad0=0, q_pos0=q_pos0, block_q=block_q, block_k=block_k,
-                 topk=topk, sink=sink, window=window, pad1=0)
+                 topk=topk, sink=sink, window=window, per_head=int(per_head))
 
 
 def set_threads(n: int = 0) -> int:
@@ -124,11 +126,12 @@ def mask(q, k, sh: Shape, units=None, with_scored=False):
     Returns (idx [n_units, 1 + cap] int32, gap [n_units] float64,
     rounds [n_units] int32) -- plus scored [n_units] int64, the candidates
     scored over all rounds, when with_scored -- units in (b, g, qb) row-major
-    order unless an explicit list of flattened unit ids is given.
+    order (g a KV head, or a query head with sh.per_head) unless an explicit
+    list of flattened unit ids is given.
     """
     lib = _load()
     q, k = _f32(q), _f32(k)
-    total = sh.batch * sh.n_kvheads * num_qblocks(sh)
+    total = sh.batch * (sh.n_qheads if sh.per_head else sh.n_kvheads) * num_qblocks(sh)
     u = None if units is None else np.ascontiguousarray(units, dtype=np.int64)
     n = total if u is None else u.size
     idx = np.empty((n, 1 + idx_cap(sh)), dtype=np.int32)

@@ -28,6 +28,10 @@
  *  - one mask per (sequence, KV head, query block); the score of a block is
  *    the max over the G*b_q query rows of the group and the b_k keys of the
  *    block of q.k, excluding keys after the row (causal) or past the range;
+ *    with per_head set (the SGLang integration's HIP_HEAD_REDUCE switch off,
+ *    "[Feature] Support Efficient Sparse HiP Attention (InfiniteHiP)"), one
+ *    mask per (sequence, query head, query block) over that head's b_q rows
+ *    and its KV head's keys, and query head h reads its own idx row;
  *  - ranking uses the raw dot q.k (a positive 1/sqrt(d) scale cannot change
  *    the order but could merge near-ties after rounding); ties go to the
  *    lower start block;
@@ -61,7 +65,7 @@ typedef struct {
   int32_t pad0;
   int64_t q_pos0;       /* absolute position of query row 0 */
   int32_t block_q, block_k, topk, sink, window;
-  int32_t pad1;
+  int32_t per_head;     /* 1: one mask per query head, not per KV-head group */
 } oracle_shape;
 
 enum { OR_OK = 0, OR_BAD = -1, OR_NOMEM = -2 };
@@ -104,6 +108,7 @@ static int shape_ok(const oracle_shape* s) {
   if (s->q_pos0 < 0 || s->q_pos0 + s->q_len > s->seq_len) return 0;
   if (s->block_q <= 0 || s->block_k <= 0 || s->topk < s->block_k) return 0;
   if (s->topk % s->block_k || s->sink < 0 || s->window < 0) return 0;
+  if (s->per_head != 0 && s->per_head != 1) return 0;
   return 1;
 }
 
@@ -136,7 +141,12 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
                      int32_t* row, double* gap_out, int32_t* rounds_out, int64_t* scored_out) {
   const int d = sh->head_dim, G = sh->n_qheads / sh->n_kvheads;
   const int64_t nqb = oracle_num_qblocks(sh), bk = sh->block_k;
-  const int64_t qb = unit % nqb, g = (unit / nqb) % sh->n_kvheads, b = unit / (nqb * sh->n_kvheads);
+  /* the mask's heads: G query heads sharing KV head g, or one query head */
+  const int64_t mh = sh->per_head ? sh->n_qheads : sh->n_kvheads;
+  const int64_t qb = unit % nqb, hm = (unit / nqb) % mh, b = unit / (nqb * mh);
+  const int64_t g = sh->per_head ? hm / G : hm;       /* KV head */
+  const int Gm = sh->per_head ? 1 : G;                 /* query heads of the mask */
+  const int64_t h0 = sh->per_head ? hm : hm * G;       /* first of them */
   const int64_t i0 = qb * sh->block_q, i1 = min64(i0 + sh->block_q, sh->q_len);
   const int64_t q_first = sh->q_pos0 + i0, q_last = sh->q_pos0 + i1 - 1;
   const int64_t Tc = min64(q_last + 1, sh->seq_len);
@@ -177,8 +187,8 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
     for (int64_t c = 0; c < nc; ++c) {
       int64_t rep = cands[c].s + (cands[c].e - cands[c].s) / 2;
       float best = -INFINITY;
-      for (int h = 0; h < G; ++h) {
-        const int64_t qh = (int64_t)g * G + h;
+      for (int h = 0; h < Gm; ++h) {
+        const int64_t qh = h0 + h;
         for (int64_t i = i0; i < i1; ++i) {
           const int64_t p = sh->q_pos0 + i;
           const float* qr = q + (((b * sh->n_qheads + qh) * sh->q_len + i) * d);
@@ -232,7 +242,8 @@ int oracle_mask(const float* q, const float* k, const oracle_shape* sh, const in
                 int64_t n_units, int32_t* idx_out, double* gap_out, int32_t* rounds_out,
                 int64_t* scored_out) {
   if (!q || !k || !idx_out || !shape_ok(sh)) return OR_BAD;
-  const int64_t total = (int64_t)sh->batch * sh->n_kvheads * oracle_num_qblocks(sh);
+  const int64_t total = (int64_t)sh->batch * (sh->per_head ? sh->n_qheads : sh->n_kvheads) *
+                        oracle_num_qblocks(sh);
   if (!units) n_units = total;
   const int64_t stride = 1 + oracle_idx_cap(sh);
   int status = OR_OK;
@@ -317,7 +328,8 @@ int oracle_attention(const float* q, const float* k, const float* v, const int32
     const int64_t i = row % sh->q_len, h = (row / sh->q_len) % sh->n_qheads;
     const int64_t b = row / ((int64_t)sh->q_len * sh->n_qheads), g = h / G;
     const int64_t p = sh->q_pos0 + i;
-    const int32_t* idx_row = idx ? idx + ((b * sh->n_kvheads + g) * nqb + i / sh->block_q) * stride : NULL;
+    const int64_t mrow = sh->per_head ? b * sh->n_qheads + h : b * sh->n_kvheads + g;  /* idx head row */
+    const int32_t* idx_row = idx ? idx + (mrow * nqb + i / sh->block_q) * stride : NULL;
     if (idx_row && (idx_row[0] < 0 || idx_row[0] > stride - 1)) {
 #pragma omp critical
       status = OR_BAD;

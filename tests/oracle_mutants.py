@@ -47,6 +47,10 @@ MUTANTS = [
     ("gqa_head", "const int64_t qh = (int64_t)g * G + h;",
      "const int64_t qh = (int64_t)g + h * sh->n_kvheads;"),
     ("stop_early", "if (longest <= 1) break;", "if (longest <= 2) break;"),
+    ("per_head_kv_map", "const int64_t g = sh->per_head ? hm / G : hm;",
+     "const int64_t g = sh->per_head ? hm % sh->n_kvheads : hm;"),
+    ("per_head_idx_row", "const int64_t mrow = sh->per_head ? b * sh->n_qheads + h : b * sh->n_kvheads + g;",
+     "const int64_t mrow = sh->per_head ? b * sh->n_qheads + g : b * sh->n_kvheads + g;"),
 ]
 
 

@@ -362,3 +362,68 @@ def test_scored_candidates_closed_form(T, bk, topk):
     n0 = topk // bk
     assert rounds[0] == int(math.log2((T // bk) // n0))
     assert scored[0] == 2 * n0 * rounds[0]
+
+
+# ---------------------------------------------------------------- per-head masks
+
+
+@pytest.mark.parametrize("kind,G,bk,topk,T", [("decode", 2, 2, 16, 200), ("decode", 4, 1, 8, 77),
+                                              ("prefill", 2, 4, 32, 150), ("prefill", 4, 2, 8, 64)])
+def test_per_head_masks_match_brute_force_per_head(kind, G, bk, topk, T):
+    # one mask per query head: each head's chunks are scored over its own rows
+    # only, against its KV head's keys (brute force on that head alone)
+    rng = np.random.default_rng(zlib.crc32(repr((kind, G, bk, topk, T)).encode()))
+    B, Hkv = 2, 2
+    Hq = Hkv * G
+    Lq = 1 if kind == "decode" else T
+    bq = 1 if kind == "decode" else 8
+    q, k = _int_inputs(rng, B, Hq, Hkv, Lq, T)
+    q_pos0 = T - Lq
+    sh = _shape(batch=B, n_qheads=Hq, n_kvheads=Hkv, head_dim=64, seq_len=T, q_len=Lq,
+                q_pos0=q_pos0, block_q=bq, block_k=bk, topk=topk, sink=bk, window=3,
+                per_head=1)
+    idx, gap, rounds = oracle.mask(q, k, sh)
+    nqb = -(-Lq // bq)
+    assert idx.shape[0] == B * Hq * nqb
+    for u in rng.choice(idx.shape[0], min(24, idx.shape[0]), replace=False):
+        b, h, qb = u // (Hq * nqb), (u // nqb) % Hq, u % nqb
+        want, want_gap, want_rounds = bf.mask_row(
+            q[:, h:h + 1], k[:, h // G:h // G + 1], b=b, g=0, qb=qb, group=1, block_q=bq,
+            block_k=bk, topk=topk, q_len=Lq, q_pos0=q_pos0, seq_len=T, sink=bk, window=3)
+        row = idx[u]
+        assert list(row[1:1 + row[0]]) == want, (u, b, h, qb)
+        assert rounds[u] == want_rounds
+
+
+def test_per_head_masks_equal_group_masks_with_one_query_head_per_kv_head():
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((1, 3, 1, 128)).astype(np.float32)
+    k = rng.standard_normal((1, 3, 500, 128)).astype(np.float32)
+    common = dict(batch=1, n_qheads=3, n_kvheads=3, head_dim=128, seq_len=500, q_len=1,
+                  q_pos0=499, block_q=1, block_k=2, topk=32, sink=4, window=8)
+    a, ga, ra = oracle.mask(q, k, _shape(per_head=0, **common))
+    b, gb, rb = oracle.mask(q, k, _shape(per_head=1, **common))
+    assert np.array_equal(a, b) and np.array_equal(ra, rb)
+
+
+def test_per_head_attention_reads_each_heads_own_row():
+    rng = np.random.default_rng(23)
+    B, Hq, Hkv, d, bk, T = 1, 4, 2, 128, 2, 300
+    q = rng.standard_normal((B, Hq, 1, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    sh = _shape(batch=B, n_qheads=Hq, n_kvheads=Hkv, head_dim=d, seq_len=T, q_len=1,
+                q_pos0=T - 1, block_q=1, block_k=bk, topk=16, sink=4, window=8, per_head=1)
+    idx, _, _ = oracle.mask(q, k, sh)
+    assert idx.shape[0] == Hq
+    out = oracle.attention(q, k, v, idx, sh).reshape(B, Hq, d)
+    for h in range(Hq):
+        g = h // 2
+        row = idx[h]
+        keys = {j for c in row[1:1 + row[0]] for j in range(c * bk, c * bk + bk) if j < T}
+        allowed = np.zeros((1, T), bool)
+        allowed[0, sorted(keys)] = True
+        ref = bf.textbook_attention(q[0, h], k[0, g], v[0, g], allowed)
+        np.testing.assert_allclose(out[0, h], ref[0], atol=2e-6, rtol=0)
+    # the two query heads of a group do pick different blocks here
+    assert not np.array_equal(idx[0], idx[1]) or not np.array_equal(idx[2], idx[3])
