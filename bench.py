@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="rotating layer buffers (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--head-masks", action="store_true",
+                    help="one mask per query head (head-reduce off) instead of per KV-head group")
     ap.add_argument("--two-calls", action="store_true",
                     help="decode: time hip_mask + hip_sparse_attn instead of hip_mask_sparse_attn")
     return ap.parse_args()
@@ -73,6 +75,20 @@ def peaks():
 
 
 # ---------------------------------------------------------------- work accounting
+
+
+HEAD_MASKS = False  # --head-masks: one mask per query head instead of per KV-head group
+
+
+def counting_view(w: W.Workload) -> W.Workload:
+    """The workload as the mask sees it: with one mask per query head, every
+    query head is its own group (for unit counts and the work counters)."""
+    return w.replace(n_kvheads=w.n_qheads) if HEAD_MASKS else w
+
+
+def oracle_layer_shape(w: W.Workload):
+    import oracle
+    return oracle.shape(head_dim=w.head_dim, per_head=int(HEAD_MASKS), **layer_shape(w))
 
 
 def layer_shape(w: W.Workload):
@@ -270,7 +286,8 @@ def reference_arm(args, w: W.Workload, world: int, rank: int):
     import oracle
     cores = oracle.set_threads(0)
     x = W.make_inputs(w)
-    sh = oracle.shape(head_dim=w.head_dim, **layer_shape(w))
+    sh = oracle_layer_shape(w)
+    w = counting_view(w)
     nqb = -(-w.q_len // w.block_q)
     units = w.batch * w.n_kvheads * nqb
     prefill = w.kind == "prefill"
@@ -329,6 +346,7 @@ def config_of(w: W.Workload, layers: int):
             "n_qheads": w.n_qheads, "n_kvheads": w.n_kvheads, "head_dim": w.head_dim,
             "topk": w.topk, "block_q": w.block_q, "block_k": w.block_k, "sink": w.sink,
             "window": w.window, "parallelism": "replicas",
+            "masks": "per query head" if HEAD_MASKS else "per KV-head group",
             "l2": f"{layers} rotating layer buffers > L2 (no flush)" if layers else None}
 
 
@@ -354,7 +372,8 @@ def cpu_baseline(w: W.Workload, x: dict, min_seconds: float = 10.0):
     (prefill, where a whole layer takes hours)."""
     import oracle
     cores = oracle.set_threads(0)
-    sh = oracle.shape(head_dim=w.head_dim, **layer_shape(w))
+    sh = oracle_layer_shape(w)
+    w = counting_view(w)
     if w.kind == "prefill":
         nqb = -(-w.q_len // w.block_q)
         units_total = w.batch * w.n_kvheads * nqb
@@ -426,6 +445,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     stream = torch.cuda.Stream(device=dev)
     shp = layer_shape(w)
     sess = hb.Session(dtype=hb.HIPS_BF16 if dt == torch.bfloat16 else hb.HIPS_F32,
+                      flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0,
                       stream=stream, **shp)
     idxs = [sess.new_idx() for _ in range(layers)]
     outs = [torch.empty_like(q0) for _ in range(layers)]
@@ -434,7 +454,8 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     # attention over it); the library runs it as one launch for bf16 groups of
     # at most 4 query rows, as the two kernels otherwise
     fused = not prefill and not args.two_calls
-    one_launch = fused and w.dtype == "bf16" and w.group * min(w.block_q, w.q_len) <= 4
+    wc = counting_view(w)
+    one_launch = fused and w.dtype == "bf16" and wc.group * min(w.block_q, w.q_len) <= 4
 
     def two_calls(l):
         hb.hip_mask(qs[l], ks[l], sess.p, idxs[l])
@@ -460,10 +481,10 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     scored = int(sess.workspace[base + 8: base + 16].cpu().numpy().view(np.uint64)[0])
     sess.check()
     idx_host = idxs[0].cpu().numpy()
-    mask_bytes = mask_algorithmic_bytes(w, scored)
-    attn_bytes = attn_algorithmic_bytes(w, idx_host, w.seq_len, w.seq_len)
-    mask_flops = mask_algorithmic_flops(w, scored)
-    attn_flops = attn_algorithmic_flops(w, idx_host) if prefill else 0
+    mask_bytes = mask_algorithmic_bytes(wc, scored)
+    attn_bytes = attn_algorithmic_bytes(wc, idx_host, w.seq_len, w.seq_len)
+    mask_flops = mask_algorithmic_flops(wc, scored)
+    attn_flops = attn_algorithmic_flops(wc, idx_host) if prefill else 0
 
     # CUDA graphs of `layers` steps (and of the remainder of K), with
     # per-kernel events in the full graph
@@ -529,7 +550,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     step_tf = (mask_flops + attn_flops) / (total_ms * 1e-3 / steps) / 1e12
     # hip_mask + hip_sparse_attn (their split merge is fused), or one launch
     launches_per_step = 1 if one_launch else 2
-    if w.dtype == "bf16" and w.group * min(w.block_q, w.q_len) > 32:
+    if w.dtype == "bf16" and wc.group * min(w.block_q, w.q_len) > 32:
         launches_per_step += 1  # the key-block norm pre-pass of a many-row mask
     two_call = None
     if fused:
@@ -691,7 +712,9 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
 
 
 def main():
+    global HEAD_MASKS
     args = parse()
+    HEAD_MASKS = args.head_masks
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         # the oracle runs on rank 0's host cores alone; no process group

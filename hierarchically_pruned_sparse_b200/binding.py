@@ -26,6 +26,7 @@ OP_MASK = 0
 OP_SPARSE = 1
 OP_DENSE = 2
 OP_MASK_SPARSE = 3
+FLAG_HEAD_MASKS = 1  # one mask per query head (idx [B, Hq, n_qblocks, row_stride])
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhip_sparse.so")
 EXPORTS = ("hip_idx_row_stride", "hip_workspace_size", "hip_workspace_init", "hip_check_status",
@@ -51,7 +52,7 @@ class Params(ctypes.Structure):
         ("dtype", ctypes.c_int32), ("q_pos0", ctypes.c_int64),
         ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("topk", ctypes.c_int32), ("sink", ctypes.c_int32),
-        ("window", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("flags", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
     ]
@@ -111,12 +112,12 @@ def _check(fn: str, code: int) -> None:
 
 def params(*, batch, n_qheads, n_kvheads, seq_len, q_len, q_pos0, dtype, block_q=1, block_k=1,
            topk=1, sink=0, window=0, mask_len=None, kv_capacity=None, head_dim=128,
-           workspace=0, workspace_bytes=0, stream=0) -> Params:
+           workspace=0, workspace_bytes=0, stream=0, flags=0) -> Params:
     return Params(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, head_dim=head_dim,
                   seq_len=seq_len, mask_len=seq_len if mask_len is None else mask_len,
                   kv_capacity=seq_len if kv_capacity is None else kv_capacity, q_len=q_len,
                   dtype=dtype, q_pos0=q_pos0, block_q=block_q, block_k=block_k, topk=topk,
-                  sink=sink, window=window, reserved=0, workspace=workspace or None,
+                  sink=sink, window=window, flags=flags, workspace=workspace or None,
                   workspace_bytes=workspace_bytes, stream=stream or None)
 
 
@@ -215,14 +216,14 @@ class Session:
 
     def __init__(self, *, batch, n_qheads, n_kvheads, seq_len, q_len, q_pos0, dtype, block_q=1,
                  block_k=1, topk=1, sink=0, window=0, mask_len=None, kv_capacity=None,
-                 stream=None):
+                 stream=None, flags=0):
         import torch
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.p = params(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, seq_len=seq_len,
                         q_len=q_len, q_pos0=q_pos0, dtype=dtype, block_q=block_q,
                         block_k=block_k, topk=topk, sink=sink, window=window,
                         mask_len=mask_len, kv_capacity=kv_capacity,
-                        stream=self.stream.cuda_stream)
+                        stream=self.stream.cuda_stream, flags=flags)
         need = max(workspace_size(self.p, op) for op in (OP_MASK, OP_SPARSE, OP_DENSE, OP_MASK_SPARSE))
         if need == 0:
             raise HipsError("hip_workspace_size", HIPS_ERR_INVALID_ARG, "invalid parameters")
@@ -245,7 +246,8 @@ class Session:
 
     def new_idx(self):
         import torch
-        return torch.empty((self.p.batch, self.p.n_kvheads, self.nqb, self.row_stride),
+        heads = self.p.n_qheads if self.p.flags & FLAG_HEAD_MASKS else self.p.n_kvheads
+        return torch.empty((self.p.batch, heads, self.nqb, self.row_stride),
                            dtype=torch.int32, device="cuda")
 
     def mask(self, q, k, idx_out=None):

@@ -33,7 +33,7 @@ int validate(const hips_params* p, int op) {
   if (p->n_qheads % p->n_kvheads) return HIPS_ERR_INVALID_ARG;
   if (p->head_dim != hips::kD) return HIPS_ERR_UNSUPPORTED;
   if (p->dtype != HIPS_F32 && p->dtype != HIPS_BF16) return HIPS_ERR_UNSUPPORTED;
-  if (p->reserved != 0) return HIPS_ERR_INVALID_ARG;
+  if (p->flags & ~HIPS_FLAG_HEAD_MASKS) return HIPS_ERR_INVALID_ARG;
   if (p->seq_len <= 0 || p->seq_len >= (int64_t{1} << 31)) return HIPS_ERR_INVALID_ARG;
   if (p->kv_capacity < p->seq_len) return HIPS_ERR_INVALID_ARG;
   if (p->q_len <= 0 || p->q_pos0 < 0 || p->q_pos0 + p->q_len > p->seq_len) return HIPS_ERR_INVALID_ARG;
@@ -56,8 +56,15 @@ int64_t row_stride(const hips_params* p) {
   return 1 + cap;
 }
 
+// One mask per query head, or one per KV-head group (the default).
+bool head_masks(const hips_params* p) { return (p->flags & HIPS_FLAG_HEAD_MASKS) != 0; }
+// Heads that own an idx row, and query heads per such head.
+int mask_heads(const hips_params* p) { return head_masks(p) ? p->n_qheads : p->n_kvheads; }
+int mask_group(const hips_params* p) { return head_masks(p) ? 1 : p->n_qheads / p->n_kvheads; }
+int kv_div(const hips_params* p) { return head_masks(p) ? p->n_qheads / p->n_kvheads : 1; }
+
 int group_rows(const hips_params* p, int block_q) {
-  return (p->n_qheads / p->n_kvheads) * std::min(block_q, p->q_len);
+  return mask_group(p) * std::min(block_q, p->q_len);
 }
 
 // ---------------------------------------------------------------- mask plan
@@ -112,8 +119,10 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   a = hips::MaskArgs{};
   a.dtype = p->dtype;
   a.n_qheads = p->n_qheads;
-  a.n_kvheads = p->n_kvheads;
-  a.group = p->n_qheads / p->n_kvheads;
+  a.n_kvheads = mask_heads(p);
+  a.group = mask_group(p);
+  a.kv_heads = p->n_kvheads;
+  a.kv_div = kv_div(p);
   a.q_len = p->q_len;
   a.block_q = p->block_q;
   a.block_k = p->block_k;
@@ -121,7 +130,7 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   a.sink = p->sink;
   a.window = p->window;
   a.nqb = static_cast<int>(cdiv(p->q_len, p->block_q));
-  a.units = static_cast<int64_t>(p->batch) * p->n_kvheads * a.nqb;
+  a.units = static_cast<int64_t>(p->batch) * mask_heads(p) * a.nqb;
   a.seq_len = p->seq_len;
   a.kv_cap = p->kv_capacity;
   a.q_pos0 = p->q_pos0;
@@ -190,7 +199,7 @@ int plan_attn_mma(const hips_params* p, bool dense, AttnPlan* plan) {
   if (p->dtype != HIPS_BF16 || a.rows_max <= 8) return HIPS_ERR_UNSUPPORTED;
   a.item_keys = dense ? 16 : p->block_k;
   if (a.item_keys > hips::attn_mma_tile_keys()) return HIPS_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(a.nqb) * p->n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(a.nqb) * a.n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
   int64_t items;
   if (dense) {
     items = cdiv(std::min<int64_t>(p->q_pos0 + p->q_len, p->seq_len), a.item_keys);
@@ -217,13 +226,17 @@ int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
   a.dtype = p->dtype;
   a.batch = p->batch;
   a.n_qheads = p->n_qheads;
-  a.n_kvheads = p->n_kvheads;
-  a.group = p->n_qheads / p->n_kvheads;
+  // a dense call has no masks: its query heads always share their KV head's tiles
+  const bool per_head = head_masks(p) && !dense;
+  a.n_kvheads = per_head ? p->n_qheads : p->n_kvheads;
+  a.group = per_head ? 1 : p->n_qheads / p->n_kvheads;
+  a.kv_heads = p->n_kvheads;
+  a.kv_div = per_head ? p->n_qheads / p->n_kvheads : 1;
   a.q_len = p->q_len;
   a.block_q = block_q;
   a.nqb = static_cast<int>(cdiv(p->q_len, block_q));
   a.dense = dense ? 1 : 0;
-  a.rows_max = group_rows(p, block_q);
+  a.rows_max = a.group * std::min(block_q, p->q_len);
   a.seq_len = p->seq_len;
   a.mask_len = dense ? p->seq_len : p->mask_len;
   a.kv_cap = p->kv_capacity;
@@ -233,7 +246,7 @@ int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
   a.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
   if (plan_attn_mma(p, dense, plan) == HIPS_OK) return HIPS_OK;
   if (a.rows_max > 8) return HIPS_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(a.nqb) * p->n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(a.nqb) * a.n_kvheads > 65535 || p->batch > 65535) return HIPS_ERR_UNSUPPORTED;
   a.item_keys = dense ? 16 : p->block_k;
   const int tile_keys = hips::attn_fma_tile_keys(p->dtype);
   if (a.item_keys > tile_keys) return HIPS_ERR_UNSUPPORTED;
@@ -244,7 +257,7 @@ int plan_attn(const hips_params* p, bool dense, AttnPlan* plan) {
   } else {
     w_max = (a.row_stride - 1) + cdiv(std::max<int64_t>(0, p->seq_len - p->mask_len), a.item_keys);
   }
-  const int64_t units = static_cast<int64_t>(p->batch) * p->n_kvheads * a.nqb;
+  const int64_t units = static_cast<int64_t>(p->batch) * a.n_kvheads * a.nqb;
   // one wave: splits x units <= SMs (one CTA per SM), at least a tile per split
   int64_t nsplit = std::min<int64_t>(kPlanSMs / units, cdiv(w_max, ipt));
   nsplit = std::max<int64_t>(1, nsplit);

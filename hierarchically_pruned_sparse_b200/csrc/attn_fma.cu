@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   };
   __syncthreads();
 
-  const size_t plane = (static_cast<size_t>(b) * a.n_kvheads + g) * static_cast<size_t>(a.kv_cap) * kRowB;
+  const size_t plane = (static_cast<size_t>(b) * a.kv_heads + g / a.kv_div) * static_cast<size_t>(a.kv_cap) * kRowB;
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) + plane;
   const unsigned char* vbase = static_cast<const unsigned char*>(a.v) + plane;
   const int ipt = kTileKeys / IK;

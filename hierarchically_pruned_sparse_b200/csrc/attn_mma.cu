@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
   const uint32_t tmem_o = tmem + 256;  // O of half h at columns 256 + 128 h
   bool timed_out = false;
 
-  const size_t plane = (static_cast<size_t>(b) * a.n_kvheads + g) * static_cast<size_t>(a.kv_cap) * 256;
+  const size_t plane = (static_cast<size_t>(b) * a.kv_heads + g / a.kv_div) * static_cast<size_t>(a.kv_cap) * 256;
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) + plane;
   const unsigned char* vbase = static_cast<const unsigned char*>(a.v) + plane;
 
@@ -196,17 +196,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
       // table lookup per row and thread
       for (int kk = lt >> 1; kk < kKeys; kk += kLoaders / 2) {
         const int item = j * ipt + (kk >> lik), kt = kk & (IK - 1);
+        int64_t key = -1;
         if (item < nitems) {
           const int2 e = table[item];
-          if (kt < e.y) {
-            const size_t row = (static_cast<size_t>(e.x) + kt) * 256;
+          if (kt < e.y) key = static_cast<int64_t>(e.x) + kt;
+        }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int ch = (lt & 1) + 2 * q;
-              const uint32_t dst = (ch >> 3) * kKVHalf + sw128_offset(kk, ch & 7);
-              cp_async16(kd + dst, kbase + row + ch * 16);
-              cp_async16(vd + dst, vbase + row + ch * 16);
-            }
+        for (int q = 0; q < 8; ++q) {
+          const int ch = (lt & 1) + 2 * q;
+          const uint32_t dst = (ch >> 3) * kKVHalf + sw128_offset(kk, ch & 7);
+          if (key >= 0) {
+            cp_async16(kd + dst, kbase + key * 256 + ch * 16);
+            cp_async16(vd + dst, vbase + key * 256 + ch * 16);
+          } else {
+            // a slot without a key: its P is 0, and 0 x V must stay 0 (the
+            // slot's stale contents could hold NaN or inf)
+            *reinterpret_cast<uint4*>(vd + dst) = make_uint4(0u, 0u, 0u, 0u);
           }
         }
       }

@@ -17,6 +17,9 @@ struct MaskArgs {
   Status* status;
   int dtype, n_qheads, n_kvheads, group, q_len, block_q, block_k, n0max, sink, window;
   int nqb, cluster, per_cta, rows_max, rows_pad, stages;
+  // K (and V) of mask head g live in head g / kv_div of kv_heads (kv_div = 1
+  // with one mask per KV-head group, = group size with one mask per query head)
+  int kv_heads, kv_div;
   int64_t units, seq_len, kv_cap, q_pos0, row_stride;
   // fused decode (tensor-core mask, few rows): when out is set, the cluster
   // of a mask row also computes the row's sparse attention over v
@@ -40,6 +43,7 @@ struct AttnArgs {
   unsigned int* counters;  // per unit, zero between calls (split merge tickets)
   int dtype, batch, n_qheads, n_kvheads, group, q_len, block_q, nqb, nsplit, dense, rows_max;
   int item_keys, table_items;
+  int kv_heads, kv_div;  // K/V of head g at head g / kv_div of kv_heads (as in MaskArgs)
   int64_t rows_total, seq_len, mask_len, kv_cap, q_pos0, row_stride;
   float scale_log2;
 };

@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   __syncthreads();
 
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
-                               (static_cast<int64_t>(b) * a.n_kvheads + g) * a.kv_cap * row_bytes<T>();
+                               (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * row_bytes<T>();
   constexpr int kRowB = row_bytes<T>();
   constexpr int kTileKeys = kTileBytes / kRowB;
   constexpr int kPasses = kTileKeys / 32;

@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
 
   const uint16_t* qg = static_cast<const uint16_t*>(a.q);
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
-                               (static_cast<int64_t>(b) * a.n_kvheads + g) * a.kv_cap * 256;
+                               (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * 256;
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   float q2max = 0.0f;
   for (int r = 0; r < N; ++r) q2max = fmaxf(q2max, qn[r]);
   const float eps_scale = kGamma * q2max;  // times |k|_2 (rounded up)
-  const int64_t knorm_base = (static_cast<int64_t>(b) * a.n_kvheads + g) * a.knorm_stride;
+  const int64_t knorm_base = (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.knorm_stride;
   const uint32_t idesc = idesc_bf16_f32(kM, N);
   const int cpt = kM >> lbk;  // candidates per tile
   int gt = 0;                 // tiles of earlier rounds (pipeline position)
@@ -944,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         const int ipt = kAK >> lbk;
         const int ntl = static_cast<int>((it1 - it0 + ipt - 1) / ipt);
         const unsigned char* vbase = static_cast<const unsigned char*>(a.v) +
-                                     (static_cast<int64_t>(b) * a.n_kvheads + g) * a.kv_cap * 256;
+                                     (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * 256;
         auto issue = [&](int t) {
           const int slot = t % S;
           unsigned char* kd = ring + slot * kTileBytes;
@@ -1010,6 +1010,10 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
             }
             load_row16<uint16_t>(kt + kk * 256, lane8, kx[u]);
             load_row16<uint16_t>(vt + kk * 256, lane8, vx[u]);
+            if (jj[u] < 0) {  // no key in this slot: stale contents must not reach o (0 x NaN)
+#pragma unroll
+              for (int e = 0; e < 16; ++e) vx[u][e] = 0.0f;
+            }
           }
           float sc[2][RC];
 #pragma unroll
@@ -1285,7 +1289,7 @@ int mask_mma_tile_keys() { return kM; }
 int mask_mma_fused_rows() { return 4; }
 
 cudaError_t launch_key_block_norms(const MaskArgs& a, int batch, cudaStream_t stream) {
-  const int64_t heads = static_cast<int64_t>(batch) * a.n_kvheads;
+  const int64_t heads = static_cast<int64_t>(batch) * a.kv_heads;
   const int64_t groups = heads * a.knorm_stride;
   const int64_t ctas = (groups + kThreads / 8 - 1) / (kThreads / 8);
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;

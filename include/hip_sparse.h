@@ -34,7 +34,8 @@
  *  - Layouts (row-major, element type = params->dtype):
  *      q, out   [batch, n_qheads, q_len, head_dim]
  *      k, v     [batch, n_kvheads, kv_capacity, head_dim]
- *      idx      int32 [batch, n_kvheads, n_qblocks, row_stride] with
+ *      idx      int32 [batch, n_kvheads, n_qblocks, row_stride] (n_qheads in
+               place of n_kvheads with HIPS_FLAG_HEAD_MASKS) with
  *               n_qblocks = ceil(q_len / block_q) and row_stride =
  *               hip_idx_row_stride(params); entry 0 of a row is nnz, then nnz
  *               ascending key-block ids, then -1 padding.
@@ -82,6 +83,17 @@ enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1 };
 
 enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2, HIPS_OP_MASK_SPARSE = 3 };
 
+/* hips_params.flags bits.
+ * HIPS_FLAG_HEAD_MASKS: one mask per query head instead of one per group of
+ *   query heads that share a KV head (the switch the SGLang integration calls
+ *   HIP_HEAD_REDUCE, here off). A head's chunks are scored over its own b_q
+ *   rows only, against its KV head's keys; idx is then
+ *   [batch, n_qheads, n_qblocks, row_stride], and query head h attends the
+ *   blocks of its own row. ("[Feature] Support Efficient Sparse HiP Attention
+ *   (InfiniteHiP)", the HIP_HEAD_REDUCE environment switch.) Dense calls
+ *   ignore it. */
+enum hips_flags { HIPS_FLAG_HEAD_MASKS = 1 };
+
 typedef struct hips_params {
   int32_t batch;      /* sequences */
   int32_t n_qheads;   /* query heads; a multiple of n_kvheads */
@@ -99,7 +111,7 @@ typedef struct hips_params {
   int32_t topk;       /* key budget k; a multiple of block_k, topk/block_k <= 2048 */
   int32_t sink;       /* leading keys always kept (0 = none) */
   int32_t window;     /* sliding-window keys always kept (0 = none) */
-  int32_t reserved;   /* must be 0 */
+  int32_t flags;      /* HIPS_FLAG_* bits; 0 for the defaults */
   void* workspace;    /* device scratch, see hip_workspace_size */
   size_t workspace_bytes;
   void* stream;       /* cudaStream_t */

@@ -104,6 +104,17 @@ def test_workspace_checked_before_launch():
     assert hb.sparse_attn_ptr(f, f, f, f, p, f) == hb.HIPS_ERR_WORKSPACE
 
 
+def test_unknown_flag_bits_rejected_and_head_masks_accepted():
+    f = 1 << 20
+    bad = _decode_params(flags=2)
+    assert hb.mask_ptr(f, f, bad, f) == hb.HIPS_ERR_INVALID_ARG
+    assert hb.workspace_size(bad, hb.OP_MASK) == 0
+    p = _decode_params(flags=hb.FLAG_HEAD_MASKS)
+    assert hb.workspace_size(p, hb.OP_MASK) >= 256
+    assert hb.idx_row_stride(p) == hb.idx_row_stride(_decode_params())
+    assert hb.mask_ptr(f, f, p, f) == hb.HIPS_ERR_WORKSPACE  # valid up to the missing workspace
+
+
 def test_fused_call_checks_on_host():
     f = 1 << 20
     need = hb.workspace_size(_decode_params(), hb.OP_MASK_SPARSE)
