@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "hip_sparse.h"
 #include "hips_common.cuh"
@@ -165,6 +166,8 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
 // device and shape (queried once, outside any stream capture in practice).
 int resident_clusters(const MaskPlan& plan) {
   struct Entry { int dev, dtype, rows, cluster, smem, n; };
+  static std::mutex mu;  // host threads may plan concurrently
+  std::lock_guard<std::mutex> lock(mu);
   static Entry cache[64];
   static int used = 0;
   int dev = 0;

@@ -21,6 +21,8 @@
 // grid is one wave (splits x units <= SM count). The kernel is launched with
 // programmatic stream serialisation: everything before the grid-dependency
 // wait (barrier set-up, query loads) overlaps the tail of the mask kernel.
+#include <mutex>
+
 #include "hips_common.cuh"
 #include "hips_kernels.h"
 
@@ -411,6 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
 template <typename T, int RC>
 cudaError_t launch_attn_t(const AttnArgs& a, int smem, cudaStream_t stream) {
   auto kern = attn_fma_kernel<T, RC>;
+  static std::mutex mu;  // host threads may launch concurrently
+  std::lock_guard<std::mutex> lock(mu);
   static int smem_set[kMaxDevices] = {};  // once per kernel and device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -28,6 +28,8 @@
 //    TMEM) when a tile's max exceeds it by more than 2^8, so P stays <= 256
 //    and the result is the exact softmax.
 // All waits are bounded; a timeout sets the status word.
+#include <mutex>
+
 #include "hips_common.cuh"
 #include "hips_kernels.h"
 #include "hips_tc.cuh"
@@ -425,6 +427,8 @@ int attn_mma_tile_keys() { return kKeys; }
 int attn_mma_rows() { return kCtaRows; }
 
 cudaError_t launch_attn_mma(const AttnArgs& a, int smem, cudaStream_t stream) {
+  static std::mutex mu;  // host threads may launch concurrently
+  std::lock_guard<std::mutex> lock(mu);
   static int smem_set[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -32,6 +32,7 @@
 //  * CTA 0 writes the idx row: sink blocks, kept blocks between sink and
 //    window, window blocks.
 #include <cooperative_groups.h>
+#include <mutex>
 
 #include "hips_common.cuh"
 #include "hips_kernels.h"
@@ -468,6 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
 template <typename T, int RC>
 cudaError_t prepare_t(const MaskArgs& a, int smem) {
   // attributes are set once per kernel and device (not inside a stream capture)
+  static std::mutex mu;  // host threads may launch concurrently
+  std::lock_guard<std::mutex> lock(mu);
   static int smem_set[kMaxDevices] = {};
   static bool big_cluster_set[kMaxDevices] = {};
   auto kern = mask_fma_kernel<T, RC>;

@@ -39,6 +39,7 @@
 //    with t_r + eps_r < max_r' (t_r' - eps_r') has s_r < s.
 #include <cooperative_groups.h>
 
+#include <mutex>
 #include <type_traits>
 
 #include "hips_common.cuh"
@@ -1211,6 +1212,8 @@ __global__ void __launch_bounds__(kThreads) key_block_norms_kernel(const unsigne
 
 template <int NC, int PER>
 cudaError_t prepare(const MaskArgs& a, int smem) {
+  static std::mutex mu;  // host threads may launch concurrently
+  std::lock_guard<std::mutex> lock(mu);
   static int smem_set[kMaxDevices] = {};
   static bool big_cluster_set[kMaxDevices] = {};
   int dev = 0;
