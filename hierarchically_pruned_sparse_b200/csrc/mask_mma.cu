@@ -341,10 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
                                (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * 256;
 
+  // With the key-norm pre-pass the read-back never touches a tile, so its
+  // ring slot is released when the tile's MMAs complete (one commit); else
+  // the four read-back warps release it after taking the norms from it.
+  const bool mma_frees_slot = a.knorm != nullptr;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], kProducers);
-      mbar_init(&empty[s], 4);
+      mbar_init(&empty[s], mma_frees_slot ? 1 : 4);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&mma_done[s], 1);
@@ -491,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
             tc_mma_bf16(tmem + tb * N, sw128_desc(a_addr), sw128_desc(b_addr), idesc, k > 0);
           }
           tc_commit(&mma_done[tb]);
+          if (mma_frees_slot) tc_commit(&empty[slot]);
         }
       }
       __syncwarp();
@@ -562,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&empty[slot]);
+          if (!mma_frees_slot) mbar_arrive(&empty[slot]);
           mbar_arrive(&tm_empty[tb]);
         }
         float eps = kvalid ? eps_scale * kn : 0.0f;
