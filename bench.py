@@ -101,17 +101,32 @@ def layer_shape(w: W.Workload):
                 kv_capacity=w.capacity)
 
 
+def elem_bytes(w: W.Workload):
+    """Bytes of a q / out element and of a k / v element."""
+    if w.dtype == "e5m2":
+        return 2, 1
+    return (2, 2) if w.dtype == "bf16" else (4, 4)
+
+
+def oracle_inputs(w: W.Workload, x: dict) -> dict:
+    """The inputs as the oracle takes them: e5m2 codes decoded by the oracle."""
+    if w.dtype != "e5m2":
+        return x
+    import oracle
+    return dict(x, k=oracle.decode_e5m2(x["k"]), v=oracle.decode_e5m2(x["v"]))
+
+
 def mask_algorithmic_bytes(w: W.Workload, scored: int) -> int:
     """Bytes the mask must read: every round reads the representative key block
     (b_k keys x d) of each candidate chunk, plus q; it writes the idx rows.
     ``scored`` is the number of candidates the kernels scored in one call
     (each candidate of each round exactly once)."""
-    esz = 2 if w.dtype == "bf16" else 4
+    esz, kv_esz = elem_bytes(w)
     units = w.batch * w.n_kvheads * (-(-w.q_len // w.block_q))
     stride = 1 + w.topk // w.block_k + -(-w.sink // w.block_k) + (
         (-(-(w.window + w.block_q - 1) // w.block_k) + 1) if w.window else 0)
     q_bytes = w.batch * w.n_qheads * w.q_len * w.head_dim * esz
-    return scored * w.block_k * w.head_dim * esz + q_bytes + units * stride * 4
+    return scored * w.block_k * w.head_dim * kv_esz + q_bytes + units * stride * 4
 
 
 def mask_algorithmic_flops(w: W.Workload, scored: int) -> int:
@@ -140,7 +155,7 @@ def attn_algorithmic_flops(w: W.Workload, idx: np.ndarray) -> int:
 def attn_algorithmic_bytes(w: W.Workload, idx: np.ndarray, seq_len: int, mask_len: int) -> int:
     """Bytes the sparse attention must read: K and V rows of every attended
     key (counted from the actual idx rows), q and idx; it writes the output."""
-    esz = 2 if w.dtype == "bf16" else 4
+    esz, kv_esz = elem_bytes(w)
     bk = w.block_k
     rows = idx.reshape(-1, idx.shape[-1])
     keys = 0
@@ -149,7 +164,7 @@ def attn_algorithmic_bytes(w: W.Workload, idx: np.ndarray, seq_len: int, mask_le
         keys += int(np.minimum(bk, mask_len - blocks * bk).clip(min=0).sum())
     keys += rows.shape[0] * max(0, seq_len - mask_len)
     qo = 2 * w.batch * w.n_qheads * w.q_len * w.head_dim * esz
-    return keys * 2 * w.head_dim * esz + qo + int(sum(int(r[0]) + 1 for r in rows)) * 4
+    return keys * 2 * w.head_dim * kv_esz + qo + int(sum(int(r[0]) + 1 for r in rows)) * 4
 
 
 # ---------------------------------------------------------------- clocks
@@ -287,7 +302,7 @@ def reference_arm(args, w: W.Workload, world: int, rank: int):
         return
     import oracle
     cores = oracle.set_threads(0)
-    x = W.make_inputs(w)
+    x = oracle_inputs(w, W.make_inputs(w))  # e5m2 codes decoded once, before timing
     sh = oracle_layer_shape(w)
     w = counting_view(w)
     nqb = -(-w.q_len // w.block_q)
@@ -349,6 +364,7 @@ def config_of(w: W.Workload, layers: int):
             "topk": w.topk, "block_q": w.block_q, "block_k": w.block_k, "sink": w.sink,
             "window": w.window, "parallelism": "replicas",
             "masks": "per query head" if HEAD_MASKS else "per KV-head group",
+            "kv_cache": {"e5m2": "fp8 e5m2 (bf16 q and out)"}.get(w.dtype, w.dtype),
             "l2": f"{layers} rotating layer buffers > L2 (no flush)" if layers else None}
 
 
@@ -374,6 +390,7 @@ def cpu_baseline(w: W.Workload, x: dict, min_seconds: float = 10.0):
     (prefill, where a whole layer takes hours)."""
     import oracle
     cores = oracle.set_threads(0)
+    x = oracle_inputs(w, x)  # e5m2 codes decoded once, before timing
     sh = oracle_layer_shape(w)
     w = counting_view(w)
     if w.kind == "prefill":
@@ -432,14 +449,15 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     x = W.make_inputs(w)
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    esz = 2 if w.dtype == "bf16" else 4
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16  # q and out
+    kt = torch.uint8 if w.dtype == "e5m2" else dt                # k and v
+    esz, kv_esz = elem_bytes(w)
     prefill = w.kind == "prefill"
-    layer_bytes = (2 * x["k"].size + x["q"][0].size) * esz
+    layer_bytes = 2 * x["k"].size * kv_esz + x["q"][0].size * esz
     layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
     layers = min(layers, 64)
-    k0 = torch.from_numpy(x["k"]).to(dev).to(dt).contiguous()
-    v0 = torch.from_numpy(x["v"]).to(dev).to(dt).contiguous()
+    k0 = torch.from_numpy(x["k"]).to(dev).to(kt).contiguous()
+    v0 = torch.from_numpy(x["v"]).to(dev).to(kt).contiguous()
     q0 = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dev).to(dt).contiguous()
     # each layer's K and V caches sit in one [2, ...] tensor, so that one copy
     # appends a new key row and value row to both
@@ -450,7 +468,8 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     qs = [q0.clone() for _ in range(layers)]
     stream = torch.cuda.Stream(device=dev)
     shp = layer_shape(w)
-    sess = hb.Session(dtype=hb.HIPS_BF16 if dt == torch.bfloat16 else hb.HIPS_F32,
+    code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
+    sess = hb.Session(dtype=code,
                       flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0,
                       stream=stream, **shp)
     idxs = [sess.new_idx() for _ in range(layers)]
@@ -461,7 +480,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     # at most 4 query rows, as the two kernels otherwise
     fused = not prefill and not args.two_calls
     wc = counting_view(w)
-    one_launch = fused and w.dtype == "bf16" and wc.group * min(w.block_q, w.q_len) <= 4
+    one_launch = fused and w.dtype != "f32" and wc.group * min(w.block_q, w.q_len) <= 4
 
     def two_calls(l, q=None):
         q = qs[l] if q is None else q
@@ -589,13 +608,17 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     # the output; captured as a graph
     e2e = None
     if not args.no_e2e and not prefill:
-        nq = q0.numel()
-        rows = np.stack([x["k"][:, :, w.seq_len - 1], x["v"][:, :, w.seq_len - 1]])
-        packed = np.concatenate([np.ascontiguousarray(x["q"][0]).reshape(-1), rows.reshape(-1)])
-        hstage = [torch.from_numpy(packed).to(dt).pin_memory() for _ in range(layers)]
-        dstage = [torch.empty(packed.size, dtype=dt, device=dev) for _ in range(layers)]
-        qv = [d[:nq].view(q0.shape) for d in dstage]
-        kvrow = [d[nq:].view(rows.shape) for d in dstage]
+        # q (as bf16/f32 bytes) then the new key and value rows (native bytes)
+        q_host = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dt).contiguous().view(torch.uint8)
+        rows = torch.from_numpy(np.ascontiguousarray(
+            np.stack([x["k"][:, :, w.seq_len - 1], x["v"][:, :, w.seq_len - 1]])))
+        rows = rows.to(kt).contiguous()
+        rb = rows.view(torch.uint8).reshape(-1)
+        packed = torch.cat([q_host.reshape(-1), rb])
+        hstage = [packed.clone().pin_memory() for _ in range(layers)]
+        dstage = [torch.empty(packed.numel(), dtype=torch.uint8, device=dev) for _ in range(layers)]
+        qv = [d[:q_host.numel()].view(dt).view(q0.shape) for d in dstage]
+        kvrow = [d[q_host.numel():].view(kt).view(rows.shape) for d in dstage]
         hout = [torch.empty(q0.shape, dtype=dt).pin_memory() for _ in range(layers)]
 
         def e2e_step(l):
@@ -630,7 +653,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
         e2.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), world)
-        h2d = packed.size * esz
+        h2d = packed.numel()
         e2e = {"value": whole_job_us_per_layer(e2e_ms, steps, world), "unit": "us/layer",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(q0.numel() * esz),
                "how": "CUDA graph per step: one H2D (pinned) of q and the new k/v rows, "
@@ -672,7 +695,7 @@ def ours(args, w: W.Workload, world: int, rank: int, local: int):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, x)
 
-    mask_kernel = "mask_mma_kernel" if w.dtype == "bf16" else "mask_fma_kernel"
+    mask_kernel = "mask_mma_kernel" if w.dtype != "f32" else "mask_fma_kernel"
     attn_kernel = "attn_mma_kernel" if prefill else "attn_fma_kernel"
     if prefill:
         dom_attn = attn_ms >= mask_ms

@@ -21,6 +21,7 @@ NOALLOC_SCRATCH_BYTES = 512 << 10
 
 HIPS_F32 = 0
 HIPS_BF16 = 1
+HIPS_BF16_E5M2 = 2  # bf16 q and out, fp8 e5m2 k and v (uint8 codes)
 
 OP_MASK = 0
 OP_SPARSE = 1

@@ -11,6 +11,10 @@
 #include "hips_common.cuh"
 #include "hips_kernels.h"
 
+static_assert(HIPS_F32 == hips::kDtypeF32 && HIPS_BF16 == hips::kDtypeBf16 &&
+                  HIPS_BF16_E5M2 == hips::kDtypeBf16E5m2,
+              "kernel dtype codes follow enum hips_dtype");
+
 namespace {
 
 thread_local int g_last_cuda_error = 0;
@@ -33,7 +37,8 @@ int validate(const hips_params* p, int op) {
   if (p->batch <= 0 || p->n_qheads <= 0 || p->n_kvheads <= 0) return HIPS_ERR_INVALID_ARG;
   if (p->n_qheads % p->n_kvheads) return HIPS_ERR_INVALID_ARG;
   if (p->head_dim != hips::kD) return HIPS_ERR_UNSUPPORTED;
-  if (p->dtype != HIPS_F32 && p->dtype != HIPS_BF16) return HIPS_ERR_UNSUPPORTED;
+  if (p->dtype != HIPS_F32 && p->dtype != HIPS_BF16 && p->dtype != HIPS_BF16_E5M2)
+    return HIPS_ERR_UNSUPPORTED;
   if (p->flags & ~HIPS_FLAG_HEAD_MASKS) return HIPS_ERR_INVALID_ARG;
   if (p->seq_len <= 0 || p->seq_len >= (int64_t{1} << 31)) return HIPS_ERR_INVALID_ARG;
   if (p->kv_capacity < p->seq_len) return HIPS_ERR_INVALID_ARG;
@@ -82,8 +87,10 @@ struct MaskPlan {
 int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   hips::MaskArgs& a = plan->a;
   const int nc = hips::mask_mma_nc(a.rows_max);
-  if (p->dtype != HIPS_BF16 || nc == 0 || p->block_k > 32 || a.units > 65535)
+  const bool kv8 = p->dtype == HIPS_BF16_E5M2;
+  if ((p->dtype != HIPS_BF16 && !kv8) || nc == 0 || p->block_k > 32 || a.units > 65535)
     return HIPS_ERR_UNSUPPORTED;
+  if (kv8 && nc != 1) return HIPS_ERR_UNSUPPORTED;  // e5m2 keys: one MMA column block
   const int cpt = hips::mask_mma_tile_keys() / p->block_k;
   const int64_t ncand = 2 * static_cast<int64_t>(a.n0max);
   // the largest cluster (any size up to the cap) with one CTA per SM for all
@@ -99,7 +106,7 @@ int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   a.per_cta = static_cast<int>(cdiv(ncand, c));
   a.rows_pad = nc * 16;
   a.stages = 0;
-  plan->smem = hips::mask_mma_smem_bytes(nc, a.n0max, a.per_cta, c);
+  plan->smem = hips::mask_mma_smem_bytes(nc, a.n0max, a.per_cta, c, kv8);
   if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
   plan->mma = true;
   plan->ws = kStatusBytes;
@@ -140,6 +147,7 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   plan->mma = false;
   plan->norms = false;
   if (plan_mask_mma(p, cluster_cap, plan) == HIPS_OK) return HIPS_OK;
+  if (p->dtype == HIPS_BF16_E5M2) return HIPS_ERR_UNSUPPORTED;  // no CUDA-core e5m2 mask
   if (a.rows_max > 32 || a.units > 65535) return HIPS_ERR_UNSUPPORTED;
   const int rc = hips::mask_fma_rc(a.rows_max);
   a.rows_pad = static_cast<int>(cdiv(a.rows_max, rc) * rc);

@@ -11,7 +11,7 @@
 //
 // Design: grid (splits, KV head x query block, sequence). Split s takes the
 // work items s, s + splits, ... (one key block each); K and V rows of a
-// 64-key tile are gathered by all threads with 16-byte cp.async copies into a
+// 64-key tile (128 keys for fp8 e5m2 rows, widened exactly when read) are gathered by all threads with 16-byte cp.async copies into a
 // 3-stage ring (all stages requested up front) (completion tracked on one mbarrier per stage), the
 // G query heads of the group share every gathered tile, and each of 8 warps
 // works on 4 keys at a time with 8 lanes per key (16 head elements per lane).
@@ -55,10 +55,12 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int tile_keys, int rc, int 
   return L;
 }
 
-template <typename T, int RC>
+// T: element type of q and out (bf16 as uint16_t, or float); KT: of k and v
+// (T, or uint8_t for fp8 e5m2 codes with bf16 q and out).
+template <typename T, typename KT, int RC>
 __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kRowB = row_bytes<T>();
+  constexpr int kRowB = row_bytes<KT>();
   constexpr int kTileKeys = kTileBytes / kRowB;
   constexpr int kPasses = kTileKeys / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
       }
       kvalid[p] = j >= 0;
       float kx[16];
-      load_row16<T>(ktile + kk * kRowB, lane8, kx);
+      load_row16<KT>(ktile + kk * kRowB, lane8, kx);
       float part[RC];
 #pragma unroll
       for (int r = 0; r < RC; ++r) {
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
       if (!kvalid[p]) continue;
       const int kk = p * 32 + warp * 4 + grp;
       float vx[16];
-      load_row16<T>(vtile + kk * kRowB, lane8, vx);
+      load_row16<KT>(vtile + kk * kRowB, lane8, vx);
       float pk[RC];
 #pragma unroll
       for (int r = 0; r < RC; ++r) pk[r] = p_sm[kk * RC + r];
@@ -410,9 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fma_kernel(AttnArgs a) {
   if (tid == 0) a.counters[unit] = 0;  // ready for the next call
 }
 
-template <typename T, int RC>
+template <typename T, typename KT, int RC>
 cudaError_t launch_attn_t(const AttnArgs& a, int smem, cudaStream_t stream) {
-  auto kern = attn_fma_kernel<T, RC>;
+  auto kern = attn_fma_kernel<T, KT, RC>;
   static std::mutex mu;  // host threads may launch concurrently
   std::lock_guard<std::mutex> lock(mu);
   static int smem_set[kMaxDevices] = {};  // once per kernel and device
@@ -438,18 +440,23 @@ cudaError_t launch_attn_t(const AttnArgs& a, int smem, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <typename T>
+template <typename T, typename KT>
 cudaError_t launch_attn_rc(const AttnArgs& a, int smem, cudaStream_t s) {
   const int R = a.rows_max;
-  if (R <= 1) return launch_attn_t<T, 1>(a, smem, s);
-  if (R <= 2) return launch_attn_t<T, 2>(a, smem, s);
-  if (R <= 4) return launch_attn_t<T, 4>(a, smem, s);
-  return launch_attn_t<T, 8>(a, smem, s);
+  if (R <= 1) return launch_attn_t<T, KT, 1>(a, smem, s);
+  if (R <= 2) return launch_attn_t<T, KT, 2>(a, smem, s);
+  if (R <= 4) return launch_attn_t<T, KT, 4>(a, smem, s);
+  return launch_attn_t<T, KT, 8>(a, smem, s);
+}
+
+// bytes of one K (V) row
+int kv_row_bytes(int dtype) {
+  return dtype == kDtypeBf16E5m2 ? kD : dtype == kDtypeBf16 ? 2 * kD : 4 * kD;
 }
 
 }  // namespace
 
-int attn_fma_tile_keys(int dtype) { return kTileBytes / (dtype == 1 ? 256 : 512); }
+int attn_fma_tile_keys(int dtype) { return kTileBytes / kv_row_bytes(dtype); }
 
 int attn_fma_smem_bytes(int dtype, int rows_max, int table_items) {
   const int rc = rows_max <= 1 ? 1 : rows_max <= 2 ? 2 : rows_max <= 4 ? 4 : 8;
@@ -457,8 +464,9 @@ int attn_fma_smem_bytes(int dtype, int rows_max, int table_items) {
 }
 
 cudaError_t launch_attn_fma(const AttnArgs& a, int smem, cudaStream_t stream) {
-  return a.dtype == 1 ? launch_attn_rc<uint16_t>(a, smem, stream)
-                      : launch_attn_rc<float>(a, smem, stream);
+  if (a.dtype == kDtypeBf16E5m2) return launch_attn_rc<uint16_t, uint8_t>(a, smem, stream);
+  return a.dtype == kDtypeBf16 ? launch_attn_rc<uint16_t, uint16_t>(a, smem, stream)
+                               : launch_attn_rc<float, float>(a, smem, stream);
 }
 
 }  // namespace hips

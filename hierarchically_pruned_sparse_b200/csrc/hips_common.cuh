@@ -13,6 +13,8 @@ constexpr int kMaxN0 = 2048;       // topk / block_k
 constexpr int kMaxDevices = 64;
 constexpr unsigned kStatusTimeout = 1u;
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
+// values of enum hips_dtype (include/hip_sparse.h)
+constexpr int kDtypeF32 = 0, kDtypeBf16 = 1, kDtypeBf16E5m2 = 2;
 
 // Status block at the head of every workspace (sticky error bits), plus the
 // number of candidate chunks the mask kernels scored since the block was
@@ -163,6 +165,53 @@ __device__ __forceinline__ void load_row16<float>(const unsigned char* row, int 
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
   x[8] = c.x; x[9] = c.y; x[10] = c.z; x[11] = c.w; x[12] = d.x; x[13] = d.y; x[14] = d.z;
   x[15] = d.w;
+}
+
+// fp8 e5m2 (1 sign, 5 exponent bits with bias 15, 2 mantissa bits; the
+// OCP 8-bit floating-point format): a code is the upper byte of the binary16
+// encoding of the same value, so widening through binary16 is exact, and so
+// is narrowing the float to bf16 afterwards (at most 3 significant bits,
+// exponents within bf16's range).
+__device__ __forceinline__ void e5m2x4_to_f32(uint32_t w, float* x) {
+  const uint32_t lo = __byte_perm(w, 0u, 0x1404);  // binary16 halves: byte 0 << 8, byte 1 << 8
+  const uint32_t hi = __byte_perm(w, 0u, 0x3424);  // byte 2 << 8, byte 3 << 8
+  asm("{\n\t.reg .b16 a, b, c, d;\n\t"
+      "mov.b32 {a, b}, %4;\n\t"
+      "mov.b32 {c, d}, %5;\n\t"
+      "cvt.f32.f16 %0, a;\n\t"
+      "cvt.f32.f16 %1, b;\n\t"
+      "cvt.f32.f16 %2, c;\n\t"
+      "cvt.f32.f16 %3, d;\n\t}"
+      : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3])
+      : "r"(lo), "r"(hi));
+}
+
+// Four e5m2 codes -> four bf16 (two words, element 0 in the low half of .x).
+__device__ __forceinline__ uint2 e5m2x4_to_bf16x4(uint32_t w) {
+  float f[4];
+  e5m2x4_to_f32(w, f);
+  return make_uint2(__byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632),
+                    __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632));
+}
+
+// One 16-byte chunk of e5m2 codes (elements 16c .. 16c + 15 of a key row) as
+// the two 16-byte bf16 chunks 2c, 2c + 1 of the row.
+__device__ __forceinline__ void e5m2x16_to_bf16(const uint4& w, uint4& c0, uint4& c1) {
+  const uint2 a = e5m2x4_to_bf16x4(w.x), b = e5m2x4_to_bf16x4(w.y);
+  const uint2 c = e5m2x4_to_bf16x4(w.z), d = e5m2x4_to_bf16x4(w.w);
+  c0 = make_uint4(a.x, a.y, b.x, b.y);
+  c1 = make_uint4(c.x, c.y, d.x, d.y);
+}
+
+template <>
+__device__ __forceinline__ void load_row16<uint8_t>(const unsigned char* row, int lane8,
+                                                    float (&x)[16]) {
+  const uint2 a = *reinterpret_cast<const uint2*>(row + lane8 * 8);
+  const uint2 b = *reinterpret_cast<const uint2*>(row + 64 + lane8 * 8);
+  e5m2x4_to_f32(a.x, x);
+  e5m2x4_to_f32(a.y, x + 4);
+  e5m2x4_to_f32(b.x, x + 8);
+  e5m2x4_to_f32(b.y, x + 12);
 }
 
 template <typename T>

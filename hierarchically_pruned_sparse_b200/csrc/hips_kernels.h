@@ -56,9 +56,10 @@ int mask_fma_tile_keys(int dtype);
 int mask_fma_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_mask_fma(const MaskArgs& a, int smem, cudaStream_t stream);
 
-// Tensor-core hierarchical top-k mask, bf16 (mask_mma.cu)
+// Tensor-core hierarchical top-k mask, bf16 keys or e5m2 keys with one MMA
+// column block (mask_mma.cu)
 int mask_mma_nc(int rows_max);  // N / 16 of the MMA (0 = too many rows)
-int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster);
+int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster, bool kv8);
 int mask_mma_tile_keys();
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream);

@@ -67,6 +67,12 @@ constexpr int kProducers = (kWarps - kProducerWarp0) * 32;
 __host__ __device__ constexpr int stages_for(int nc, int per) {
   return per > 8 ? 2 : nc >= 8 ? 3 : 4;
 }
+// fp8 e5m2 keys: the producers land raw rows (128 bytes) in two staging
+// tiles and widen them into the ring, which gives up a slot for the staging
+constexpr int kRawTileBytes = kM * 128;
+__host__ __device__ constexpr int ring_stages(int nc, int per, bool kv8) {
+  return kv8 ? (stages_for(nc, per) > 2 ? stages_for(nc, per) - 1 : 2) : stages_for(nc, per);
+}
 // Many-row masks keep the arrays that only the selection uses (histogram,
 // band lists, keep flags, row marks) in the last ring slot, which the
 // selection never needs: that is what makes room for the slot.
@@ -75,7 +81,7 @@ __host__ __device__ constexpr int tmem_cols_for(int nc) { return nc * 32 < 32 ? 
 __host__ __device__ constexpr int mask_words(int nc) { return nc < 2 ? 1 : nc / 2; }
 
 struct MmaSmem {
-  int ring, bq, bar, slot, rpos, qn, cs, ce, keepb, band, band_key, xch, hist, rowmask, vmask,
+  int ring, raw, bq, bar, slot, rpos, qn, cs, ce, keepb, band, band_key, xch, hist, rowmask, vmask,
       scratch, total;
 };
 
@@ -85,12 +91,13 @@ __host__ __device__ inline int al(int x, int a) { return (x + a - 1) / a * a; }
 // copy and writes the next round's list into the other. xch holds the (score,
 // bound) of every candidate of a round: each CTA writes its own candidates
 // into every CTA of the cluster; two copies alternate between rounds.
-__host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cluster) {
+__host__ __device__ inline MmaSmem mma_layout(int nc, int per, int n0max, int cluster, bool kv8) {
   MmaSmem L;
   const int n = (2 * n0max + 3) & ~3;  // candidate buffer stride (16-byte rows of 4)
-  const int S = stages_for(nc, per);
+  const int S = ring_stages(nc, per, kv8);
   int o = 0;
   L.ring = o;     o += S * kTileBytes;
+  L.raw = o;      o += kv8 ? 2 * kRawTileBytes : 0;
   L.bq = o;       o += nc * 16 * 256;
   L.bar = o;      o += al(8 * (3 * S + 5), 16);  // every region below starts on 16 bytes
   L.slot = o;     o += 16;
@@ -282,10 +289,42 @@ __device__ __forceinline__ void gather_tile(unsigned char* tile, const unsigned 
   }
 }
 
-template <int NC, int PER>
+// Widen the e5m2 chunk c (of 8) of tile key kk into bf16 chunks 2c, 2c + 1
+// of the swizzled tile.
+__device__ __forceinline__ void store_e5m2_chunk(unsigned char* tile, int kk, int c, const uint4& w) {
+  uint4 c0, c1;
+  e5m2x16_to_bf16(w, c0, c1);
+  const int ch = 2 * c;
+  *reinterpret_cast<uint4*>(tile + (ch >> 3) * kHalfBytes + sw128_offset(kk, ch & 7)) = c0;
+  *reinterpret_cast<uint4*>(tile + ((ch + 1) >> 3) * kHalfBytes + sw128_offset(kk, (ch + 1) & 7)) = c1;
+}
+
+// gather_tile for e5m2 key rows (128 bytes), widened to bf16 on the way:
+// thread p of nthr loads chunks (p & 1) + 2i of key p / 2 (+ nthr / 2, ...).
+template <typename KeyOf>
+__device__ __forceinline__ void gather_tile_e5m2(unsigned char* tile, const unsigned char* kbase,
+                                                 int nkeys, int p, int nthr, int64_t Tc,
+                                                 KeyOf key_of) {
+  for (int kk = p >> 1; kk < nkeys; kk += nthr >> 1) {
+    const int64_t j = key_of(kk);
+    if (j < Tc) {
+      const uint4* src = reinterpret_cast<const uint4*>(kbase + j * 128);
+      uint4 w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = __ldg(src + (p & 1) + 2 * i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) store_e5m2_chunk(tile, kk, (p & 1) + 2 * i, w[i]);
+    }
+  }
+}
+
+// KV8: k and v hold fp8 e5m2 codes (q and out stay bf16).
+template <int NC, int PER, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   constexpr int N = NC * 16;
-  constexpr int S = stages_for(NC, PER);
+  constexpr int S = ring_stages(NC, PER, KV8);
+  constexpr int kRowB = KV8 ? 128 : 256;  // bytes of a K (V) row
+  using KvT = std::conditional_t<KV8, uint8_t, uint16_t>;
   constexpr int TCOLS = tmem_cols_for(NC);
   constexpr int MW = mask_words(NC);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -311,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   const int per_cta = a.per_cta;
   const int nbuf = (2 * a.n0max + 3) & ~3;  // stride between the two candidate buffers
 
-  const MmaSmem L = mma_layout(NC, PER, a.n0max, C);
+  const MmaSmem L = mma_layout(NC, PER, a.n0max, C, KV8);
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   unsigned char* ring = smem + L.ring;
   unsigned char* bq = smem + L.bq;
@@ -339,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
 
   const uint16_t* qg = static_cast<const uint16_t*>(a.q);
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k) +
-                               (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * 256;
+                               (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * kRowB;
 
   // With the key-norm pre-pass the read-back never touches a tile, so its
   // ring slot is released when the tile's MMAs complete (one commit); else
@@ -469,14 +508,70 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducers / 32) {
       // ---------------- gather tiles into the ring
       const int p = tid - kProducerWarp0 * 32;
-      for (int t = 0; t < ntiles; ++t) {
-        const int gi = gt + t, slot = gi % S;
-        if (gi >= S && !timed_out && !mbar_wait(&empty[slot], ((gi / S) - 1) & 1)) timed_out = true;
-        const int cf = c_lo + t * cpt;
-        const int nkeys = min(cpt, c_hi - cf) << lbk;
-        gather_tile(ring + slot * kTileBytes, kbase, nkeys, p, kProducers, Tc,
-                    [&](int kk) { return rep_key(cf + (kk >> lbk)) + (kk & (bk - 1)); });
-        cp_async_arrive(&full[slot]);
+      if constexpr (KV8) {
+        // raw e5m2 rows of tile t land in staging tile gi & 1 (cp.async) while
+        // this thread widens its own chunks of tile t - 1 into the ring; thread
+        // p handles chunks (p & 1) + 2i of keys p / 2, p / 2 + 48, ...
+        unsigned char* raw = smem + L.raw;
+        auto key_at = [&](int t, int kk) -> int64_t {
+          const int cf = c_lo + t * cpt;
+          return rep_key(cf + (kk >> lbk)) + (kk & (bk - 1));
+        };
+        auto nkeys_of = [&](int t) { return min(cpt, c_hi - (c_lo + t * cpt)) << lbk; };
+        auto land = [&](int t) {
+          unsigned char* dst = raw + ((gt + t) & 1) * kRawTileBytes;
+          const int nkeys = nkeys_of(t);
+          for (int kk = p >> 1; kk < nkeys; kk += kProducers >> 1) {
+            const int64_t j = key_at(t, kk);
+            if (j < Tc) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int c = (p & 1) + 2 * i;
+                cp_async16(dst + kk * 128 + c * 16, kbase + j * 128 + c * 16);
+              }
+            }
+          }
+          cp_async_commit();
+        };
+        auto widen = [&](int t) {  // this thread's chunks of tile t have landed
+          const int gi = gt + t, slot = gi % S;
+          if (gi >= S && !timed_out && !mbar_wait(&empty[slot], ((gi / S) - 1) & 1)) timed_out = true;
+          const unsigned char* src = raw + (gi & 1) * kRawTileBytes;
+          unsigned char* tile = ring + slot * kTileBytes;
+          const int nkeys = nkeys_of(t);
+          for (int kk = p >> 1; kk < nkeys; kk += kProducers >> 1) {
+            if (key_at(t, kk) < Tc) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int c = (p & 1) + 2 * i;
+                store_e5m2_chunk(tile, kk, c, *reinterpret_cast<const uint4*>(src + kk * 128 + c * 16));
+              }
+            }
+          }
+          fence_proxy_async_smem();  // generic writes -> tensor-core reads
+          mbar_arrive(&full[slot]);
+        };
+        for (int t = 0; t < ntiles; ++t) {
+          land(t);
+          if (t >= 1) {
+            cp_async_wait<1>();
+            widen(t - 1);
+          }
+        }
+        if (ntiles >= 1) {
+          cp_async_wait<0>();
+          widen(ntiles - 1);
+        }
+      } else {
+        for (int t = 0; t < ntiles; ++t) {
+          const int gi = gt + t, slot = gi % S;
+          if (gi >= S && !timed_out && !mbar_wait(&empty[slot], ((gi / S) - 1) & 1)) timed_out = true;
+          const int cf = c_lo + t * cpt;
+          const int nkeys = min(cpt, c_hi - cf) << lbk;
+          gather_tile(ring + slot * kTileBytes, kbase, nkeys, p, kProducers, Tc,
+                      [&](int kk) { return rep_key(cf + (kk >> lbk)) + (kk & (bk - 1)); });
+          cp_async_arrive(&full[slot]);
+        }
       }
     } else if (warp == kIssuerWarp) {
       // ---------------- MMA issue (one thread)
@@ -720,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         const int64_t j = rep_key(ci) + kt;
         const bool jok = live && j < Tc;
         float kx[16];
-        load_row16<uint16_t>(kbase + (jok ? j : 0) * 256, lane8, kx);
+        load_row16<KvT>(kbase + (jok ? j : 0) * kRowB, lane8, kx);
         float part[8];
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) {
@@ -748,8 +843,11 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
       for (int m0 = 0; m0 < nband; m0 += bpt) {
         const int mcnt = min(bpt, nband - m0);
         const int nkeys = mcnt << lbk;
-        gather_tile(tile, kbase, nkeys, tid, kThreads, Tc,
-                    [&](int kk) { return rep_key(band[m0 + (kk >> lbk)]) + (kk & (bk - 1)); });
+        auto band_key_of = [&](int kk) { return rep_key(band[m0 + (kk >> lbk)]) + (kk & (bk - 1)); };
+        if constexpr (KV8)
+          gather_tile_e5m2(tile, kbase, nkeys, tid, kThreads, Tc, band_key_of);
+        else
+          gather_tile(tile, kbase, nkeys, tid, kThreads, Tc, band_key_of);
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async_smem();
@@ -950,19 +1048,20 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
         const int ipt = kAK >> lbk;
         const int ntl = static_cast<int>((it1 - it0 + ipt - 1) / ipt);
         const unsigned char* vbase = static_cast<const unsigned char*>(a.v) +
-                                     (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * 256;
+                                     (static_cast<int64_t>(b) * a.kv_heads + g / a.kv_div) * a.kv_cap * kRowB;
+        constexpr int kChunks = kRowB / 16;  // 16-byte chunks of a K (V) row
         auto issue = [&](int t) {
           const int slot = t % S;
           unsigned char* kd = ring + slot * kTileBytes;
           unsigned char* vd = kd + kHalfBytes;
           const int64_t f = it0 + static_cast<int64_t>(t) * ipt;
           const int nk = static_cast<int>(min64(ipt, it1 - f)) << lbk;
-          for (int i = tid; i < nk * 16; i += kThreads) {
-            const int kk = i >> 4, ch = i & 15;
+          for (int i = tid; i < nk * kChunks; i += kThreads) {
+            const int kk = i / kChunks, ch = i % kChunks;
             const int64_t j = (block_at(f + (kk >> lbk)) << lbk) + (kk & (bk - 1));
             if (j < Tc) {
-              cp_async16(kd + kk * 256 + ch * 16, kbase + j * 256 + ch * 16);
-              cp_async16(vd + kk * 256 + ch * 16, vbase + j * 256 + ch * 16);
+              cp_async16(kd + kk * kRowB + ch * 16, kbase + j * kRowB + ch * 16);
+              cp_async16(vd + kk * kRowB + ch * 16, vbase + j * kRowB + ch * 16);
             }
           }
           cp_async_arrive(&abar[slot]);
@@ -1014,8 +1113,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
               const int64_t j = (block_at(f + (kk >> lbk)) << lbk) + (kk & (bk - 1));
               jj[u] = j < Tc ? j : -1;
             }
-            load_row16<uint16_t>(kt + kk * 256, lane8, kx[u]);
-            load_row16<uint16_t>(vt + kk * 256, lane8, vx[u]);
+            load_row16<KvT>(kt + kk * kRowB, lane8, kx[u]);
+            load_row16<KvT>(vt + kk * kRowB, lane8, vx[u]);
             if (jj[u] < 0) {  // no key in this slot: stale contents must not reach o (0 x NaN)
 #pragma unroll
               for (int e = 0; e < 16; ++e) vx[u][e] = 0.0f;
@@ -1215,7 +1314,7 @@ __global__ void __launch_bounds__(kThreads) key_block_norms_kernel(const unsigne
   if (lane8 == 0) out[gid] = sqrtf(m) * kNormUp;
 }
 
-template <int NC, int PER>
+template <int NC, int PER, bool KV8>
 cudaError_t prepare(const MaskArgs& a, int smem) {
   static std::mutex mu;  // host threads may launch concurrently
   std::lock_guard<std::mutex> lock(mu);
@@ -1226,19 +1325,19 @@ cudaError_t prepare(const MaskArgs& a, int smem) {
   if (e != cudaSuccess) return e;
   dev %= kMaxDevices;
   if (smem > smem_set[dev]) {
-    e = cudaFuncSetAttribute(mask_mma_kernel<NC, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(mask_mma_kernel<NC, PER, KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     smem_set[dev] = smem;
   }
   if (a.cluster > 8 && !big_cluster_set[dev]) {
-    e = cudaFuncSetAttribute(mask_mma_kernel<NC, PER>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(mask_mma_kernel<NC, PER, KV8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     big_cluster_set[dev] = true;
   }
   return cudaSuccess;
 }
 
-template <int NC, int PER>
+template <int NC, int PER, bool KV8>
 cudaLaunchConfig_t make_config(const MaskArgs& a, int smem, cudaStream_t stream,
                                cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
@@ -1255,25 +1354,25 @@ cudaLaunchConfig_t make_config(const MaskArgs& a, int smem, cudaStream_t stream,
   return cfg;
 }
 
-template <int NC, int PER>
+template <int NC, int PER, bool KV8>
 cudaError_t launch_nc(const MaskArgs& a, int smem, cudaStream_t stream) {
-  cudaError_t e = prepare<NC, PER>(a, smem);
+  cudaError_t e = prepare<NC, PER, KV8>(a, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_config<NC, PER>(a, smem, stream, attr);
-  return cudaLaunchKernelEx(&cfg, mask_mma_kernel<NC, PER>, a);
+  cudaLaunchConfig_t cfg = make_config<NC, PER, KV8>(a, smem, stream, attr);
+  return cudaLaunchKernelEx(&cfg, mask_mma_kernel<NC, PER, KV8>, a);
 }
 
-template <int NC, int PER>
+template <int NC, int PER, bool KV8>
 int resident_nc(const MaskArgs& a, int smem) {
-  if (prepare<NC, PER>(a, smem) != cudaSuccess) {
+  if (prepare<NC, PER, KV8>(a, smem) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
   }
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_config<NC, PER>(a, smem, nullptr, attr);
+  cudaLaunchConfig_t cfg = make_config<NC, PER, KV8>(a, smem, nullptr, attr);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, mask_mma_kernel<NC, PER>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, mask_mma_kernel<NC, PER, KV8>, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
   }
@@ -1287,9 +1386,9 @@ int mask_mma_nc(int rows_max) {
   return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : n <= 8 ? 8 : n <= 16 ? 16 : 0;
 }
 
-int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster) {
+int mask_mma_smem_bytes(int nc, int n0max, int per_cta, int cluster, bool kv8) {
   (void)per_cta;
-  return mma_layout(nc, n0max <= 1024 ? 8 : 16, n0max, cluster).total;
+  return mma_layout(nc, n0max <= 1024 ? 8 : 16, n0max, cluster, kv8).total;
 }
 
 int mask_mma_tile_keys() { return kM; }
@@ -1308,23 +1407,33 @@ cudaError_t launch_key_block_norms(const MaskArgs& a, int batch, cudaStream_t st
 }
 
 int mask_mma_max_active_clusters(const MaskArgs& a, int smem) {
+  const bool p16 = a.n0max > 1024;
+  if (a.dtype == kDtypeBf16E5m2) {  // one MMA column block only
+    if (mask_mma_nc(a.rows_max) != 1) return -1;
+    return p16 ? resident_nc<1, 16, true>(a, smem) : resident_nc<1, 8, true>(a, smem);
+  }
   switch (mask_mma_nc(a.rows_max)) {
-    case 1: return a.n0max <= 1024 ? resident_nc<1, 8>(a, smem) : resident_nc<1, 16>(a, smem);
-    case 2: return a.n0max <= 1024 ? resident_nc<2, 8>(a, smem) : resident_nc<2, 16>(a, smem);
-    case 4: return a.n0max <= 1024 ? resident_nc<4, 8>(a, smem) : resident_nc<4, 16>(a, smem);
-    case 8: return a.n0max <= 1024 ? resident_nc<8, 8>(a, smem) : resident_nc<8, 16>(a, smem);
-    case 16: return a.n0max <= 1024 ? resident_nc<16, 8>(a, smem) : resident_nc<16, 16>(a, smem);
+    case 1: return p16 ? resident_nc<1, 16, false>(a, smem) : resident_nc<1, 8, false>(a, smem);
+    case 2: return p16 ? resident_nc<2, 16, false>(a, smem) : resident_nc<2, 8, false>(a, smem);
+    case 4: return p16 ? resident_nc<4, 16, false>(a, smem) : resident_nc<4, 8, false>(a, smem);
+    case 8: return p16 ? resident_nc<8, 16, false>(a, smem) : resident_nc<8, 8, false>(a, smem);
+    case 16: return p16 ? resident_nc<16, 16, false>(a, smem) : resident_nc<16, 8, false>(a, smem);
     default: return -1;
   }
 }
 
 cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream) {
+  const bool p16 = a.n0max > 1024;
+  if (a.dtype == kDtypeBf16E5m2) {
+    if (mask_mma_nc(a.rows_max) != 1) return cudaErrorInvalidValue;
+    return p16 ? launch_nc<1, 16, true>(a, smem, stream) : launch_nc<1, 8, true>(a, smem, stream);
+  }
   switch (mask_mma_nc(a.rows_max)) {
-    case 1: return a.n0max <= 1024 ? launch_nc<1, 8>(a, smem, stream) : launch_nc<1, 16>(a, smem, stream);
-    case 2: return a.n0max <= 1024 ? launch_nc<2, 8>(a, smem, stream) : launch_nc<2, 16>(a, smem, stream);
-    case 4: return a.n0max <= 1024 ? launch_nc<4, 8>(a, smem, stream) : launch_nc<4, 16>(a, smem, stream);
-    case 8: return a.n0max <= 1024 ? launch_nc<8, 8>(a, smem, stream) : launch_nc<8, 16>(a, smem, stream);
-    case 16: return a.n0max <= 1024 ? launch_nc<16, 8>(a, smem, stream) : launch_nc<16, 16>(a, smem, stream);
+    case 1: return p16 ? launch_nc<1, 16, false>(a, smem, stream) : launch_nc<1, 8, false>(a, smem, stream);
+    case 2: return p16 ? launch_nc<2, 16, false>(a, smem, stream) : launch_nc<2, 8, false>(a, smem, stream);
+    case 4: return p16 ? launch_nc<4, 16, false>(a, smem, stream) : launch_nc<4, 8, false>(a, smem, stream);
+    case 8: return p16 ? launch_nc<8, 16, false>(a, smem, stream) : launch_nc<8, 8, false>(a, smem, stream);
+    case 16: return p16 ? launch_nc<16, 16, false>(a, smem, stream) : launch_nc<16, 8, false>(a, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -24,6 +24,9 @@ for them):
   the draws of one head are taken in [dim][t] order.
 * bf16 workloads round every tensor to bf16 (round to nearest even) after
   drawing; the float32 arrays returned hold exactly the bf16 values.
+* e5m2 workloads (an fp8 KV cache) round q to bf16 and return k and v as
+  uint8 fp8 e5m2 codes of the bf16 values, each rounded once to the nearest
+  e5m2 value (ties to even). Needles are coded the same way.
 """
 from __future__ import annotations
 
@@ -61,7 +64,7 @@ class Workload:
     topk: int
     sink: int
     window: int
-    dtype: str  # "f32" | "bf16"
+    dtype: str  # "f32" | "bf16" | "e5m2" (bf16 q, fp8 e5m2 k and v)
     needles: int = 0  # per KV head
     needle_mode: str = "none"  # "uniform" | "loguniform" | "none"
     refresh: int = 1  # decode steps served by one mask (r_m)
@@ -98,8 +101,11 @@ DECODE_B16_REUSE = Workload("decode_B16_T128k_h32x8_bf16_rm8", "decode", 16, 32,
 DECODE_1M = Workload("decode_T1M_h32x8_bf16", "decode", 1, 32, 8, 128, 1048576,
                      1, 4, 4096, 256, 2048, "bf16", needles=64, needle_mode="loguniform")
 
+# the 128k decode step over an fp8 e5m2 KV cache (bf16 queries)
+DECODE_128K_E5M2 = dataclasses.replace(DECODE_128K, name="decode_T128k_h32x8_e5m2", dtype="e5m2")
+
 WORKLOADS = {w.name: w for w in (DECODE_8K_F32, DECODE_128K, PREFILL_32K,
-                                 DECODE_B16_REUSE, DECODE_1M)}
+                                 DECODE_B16_REUSE, DECODE_1M, DECODE_128K_E5M2)}
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
@@ -112,6 +118,21 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     """The upper 16 bits of bf16-exact float32 values, as uint16."""
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
     return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def e5m2_codes(x: np.ndarray) -> np.ndarray:
+    """fp8 e5m2 codes (uint8) of float32 values, rounded once to the nearest
+    e5m2 value (ties to even): 2 mantissa bits kept on the float32 encoding,
+    multiples of 2^-16 below 2^-14 (the subnormals). The rounded value is
+    exact in binary16, whose encoding's upper byte is the code. Values must
+    stay below the e5m2 range limit."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    r = (u + np.uint32(0xFFFFF) + ((u >> np.uint32(21)) & np.uint32(1))) & np.uint32(0xFFE00000)
+    y = r.view(np.float32).copy()
+    small = np.abs(x) < np.float32(2.0 ** -14)
+    y[small] = (np.rint(x[small].astype(np.float64) * 2.0 ** 16) / 2.0 ** 16).astype(np.float32)
+    return (y.astype(np.float16).view(np.uint16) >> np.uint16(8)).astype(np.uint8)
 
 
 def _ar1(rng: np.random.Generator, heads: int, length: int, dim: int) -> np.ndarray:
@@ -151,7 +172,8 @@ def _needle_positions(rng: np.random.Generator, w: Workload, count: int, qpos: i
 def make_sequence(w: Workload, b: int = 0) -> dict:
     """Inputs of batch entry ``b`` (seed ``w.seed + b``).
 
-    Returns float32 arrays ``k``/``v`` [Hkv, capacity, d] and ``q``
+    Returns float32 arrays ``k``/``v`` [Hkv, capacity, d] (uint8 e5m2 codes
+    for e5m2 workloads) and ``q``
     [steps, Hq, Lq, d] (steps = ``refresh`` for decode, 1 for prefill), plus
     ``needle_pos`` [Hkv, needles].
     """
@@ -163,7 +185,7 @@ def make_sequence(w: Workload, b: int = 0) -> dict:
         q = rng.standard_normal((w.refresh, hq, 1, d), dtype=np.float32)
     else:
         q = _ar1(rng, hq, w.seq_len, d)[None]
-    if w.dtype == "bf16":
+    if w.dtype in ("bf16", "e5m2"):
         k, v, q = bf16_round(k), bf16_round(v), bf16_round(q)
     needle_pos = np.zeros((hkv, w.needles), dtype=np.int64)
     if w.needles:
@@ -177,8 +199,10 @@ def make_sequence(w: Workload, b: int = 0) -> dict:
             for j in range(w.needles):
                 qv = q[0, h * g + (j % g), 0]
                 key = NEEDLE_GAIN * qv / np.float32(np.linalg.norm(qv)) + NEEDLE_NOISE * noise[j]
-                k[h, pos[j]] = bf16_round(key) if w.dtype == "bf16" else key
+                k[h, pos[j]] = bf16_round(key) if w.dtype in ("bf16", "e5m2") else key
             needle_pos[h] = pos
+    if w.dtype == "e5m2":
+        k, v = e5m2_codes(k), e5m2_codes(v)
     return {"q": q, "k": k, "v": v, "needle_pos": needle_pos}
 
 

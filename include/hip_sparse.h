@@ -31,11 +31,12 @@
  *    never frees or keeps them. Calls are asynchronous on params->stream
  *    (a cudaStream_t; NULL is the legacy default stream), allocate nothing,
  *    and never synchronise the device.
- *  - Layouts (row-major, element type = params->dtype):
+ *  - Layouts (row-major, element type = params->dtype; with HIPS_BF16_E5M2
+ *    k and v hold 1-byte e5m2 codes and q, out bf16):
  *      q, out   [batch, n_qheads, q_len, head_dim]
  *      k, v     [batch, n_kvheads, kv_capacity, head_dim]
  *      idx      int32 [batch, n_kvheads, n_qblocks, row_stride] (n_qheads in
-               place of n_kvheads with HIPS_FLAG_HEAD_MASKS) with
+ *               place of n_kvheads with HIPS_FLAG_HEAD_MASKS) with
  *               n_qblocks = ceil(q_len / block_q) and row_stride =
  *               hip_idx_row_stride(params); entry 0 of a row is nnz, then nnz
  *               ascending key-block ids, then -1 padding.
@@ -79,7 +80,17 @@ enum hips_status {
   HIPS_ERR_TOO_LARGE = -6    /* more scratch than hip_sparse_attn_noalloc's fixed array */
 };
 
-enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1 };
+/* Element types. HIPS_BF16_E5M2 is an fp8 KV cache: k and v hold fp8 e5m2
+ * codes (1 byte per element; the OCP 8-bit floating-point format, the KV
+ * cache type of "--kv-cache-dtype fp8_e5m2" in the HiP attention serving
+ * command of the SGLang pull request "[Feature] Support Efficient Sparse HiP
+ * Attention (InfiniteHiP)"), while q and out are bf16. Every code widens
+ * exactly to bf16, and the mask and attention are those of bf16 keys and
+ * values with the widened values. Supported for masks of at most 16 query
+ * rows (decode: G heads x b_q <= 16) with block_k <= 32, and for attention
+ * of at most 8 rows per query block; other shapes return
+ * HIPS_ERR_UNSUPPORTED. */
+enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1, HIPS_BF16_E5M2 = 2 };
 
 enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2, HIPS_OP_MASK_SPARSE = 3 };
 
@@ -105,6 +116,7 @@ typedef struct hips_params {
   int64_t kv_capacity;/* allocated length of the key axis, >= seq_len */
   int32_t q_len;      /* query rows per sequence: 1 for decode, T for prefill */
   int32_t dtype;      /* enum hips_dtype of q, k, v and out (accumulation is fp32) */
+                      /* (HIPS_BF16_E5M2: q, out bf16; k, v e5m2) */
   int64_t q_pos0;     /* absolute position of query row 0; q_pos0 + q_len <= seq_len */
   int32_t block_q;    /* query rows sharing one mask (b_q) */
   int32_t block_k;    /* keys per block (b_k), a power of two */

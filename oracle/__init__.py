@@ -74,6 +74,8 @@ def _load():
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_mask.restype = ctypes.c_int
     lib.oracle_mask.argtypes = [f32p, f32p, P(Shape), i64p, ctypes.c_int64, i32p, f64p, i32p, i64p]
+    lib.oracle_decode_e5m2.restype = None
+    lib.oracle_decode_e5m2.argtypes = [P(ctypes.c_uint8), ctypes.c_int64, f32p]
     lib.oracle_attention.restype = ctypes.c_int
     lib.oracle_attention.argtypes = [f32p, f32p, f32p, i32p, P(Shape), i64p, ctypes.c_int64, f32p]
     _lib = lib
@@ -102,6 +104,14 @@ def shape(*, batch, n_qheads, n_kvheads, head_dim, seq_len, q_len, q_pos0, block
 def set_threads(n: int = 0) -> int:
     """Set the OpenMP thread count (n <= 0 keeps it); returns the count in use."""
     return int(_load().oracle_set_threads(int(n)))
+
+
+def decode_e5m2(codes) -> np.ndarray:
+    """float32 values of fp8 e5m2 codes (uint8 array of any shape)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float32)
+    _load().oracle_decode_e5m2(_ptr(c, ctypes.c_uint8), c.size, _ptr(out, ctypes.c_float))
+    return out
 
 
 def canonical_dot(q, k) -> np.float32:

@@ -19,6 +19,14 @@
  *            summary): Approach (centre tokens as chunk representatives),
  *            Measured effects ("Add V 2k and D 1k": always-kept sink and
  *            sliding-window blocks), Limitations (mask refresh interval r_m).
+ *  [PR]      "[Feature] Support Efficient Sparse HiP Attention (InfiniteHiP)"
+ *            (SGLang pull request): the serving commands run HiP attention
+ *            over a KV cache stored as fp8 e5m2 (--kv-cache-dtype
+ *            fp8_e5m2). The code values follow the published 8-bit
+ *            floating-point format (OCP "8-bit Floating Point
+ *            Specification", E5M2): 1 sign bit, 5 exponent bits with bias 15,
+ *            2 mantissa bits; exponent 0 holds zero and the subnormals
+ *            m/4 * 2^-14, exponent 31 the infinities (m = 0) and NaNs.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - chunk i of n0 over N blocks is [floor(iN/n0), floor((i+1)N/n0));
@@ -82,6 +90,26 @@ int oracle_set_threads(int n) {
   (void)n;
   return 1;
 #endif
+}
+
+/* Value of one fp8 e5m2 code ([PR]; format definition in the header). */
+static double e5m2_value(uint8_t c) {
+  const int sign = c >> 7, e = (c >> 2) & 31, m = c & 3;
+  double v;
+  if (e == 0)
+    v = ldexp(m / 4.0, -14);
+  else if (e == 31)
+    v = m == 0 ? INFINITY : NAN;
+  else
+    v = ldexp(1.0 + m / 4.0, e - 15);
+  return sign ? -v : v;
+}
+
+/* Decode n e5m2 codes to float (every finite code is exact in float). An
+ * fp8 KV cache is attended with these values: the mask and the attention
+ * below then take them like any other keys and values. */
+void oracle_decode_e5m2(const uint8_t* codes, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = (float)e5m2_value(codes[i]);
 }
 
 /* The fp32 dot in the canonical order described in the header. */

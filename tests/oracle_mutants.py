@@ -51,6 +51,10 @@ MUTANTS = [
      "const int64_t g = sh->per_head ? hm % sh->n_kvheads : hm;"),
     ("per_head_idx_row", "const int64_t mrow = sh->per_head ? b * sh->n_qheads + h : b * sh->n_kvheads + g;",
      "const int64_t mrow = sh->per_head ? b * sh->n_qheads + g : b * sh->n_kvheads + g;"),
+    ("e5m2_bias", "v = ldexp(1.0 + m / 4.0, e - 15);", "v = ldexp(1.0 + m / 4.0, e - 16);"),
+    ("e5m2_subnormal", "v = ldexp(m / 4.0, -14);", "v = ldexp(1.0 + m / 4.0, -15);"),
+    ("e5m2_mantissa", "const int sign = c >> 7, e = (c >> 2) & 31, m = c & 3;",
+     "const int sign = c >> 7, e = (c >> 2) & 31, m = (c >> 1) & 3;"),
 ]
 
 

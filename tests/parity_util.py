@@ -11,18 +11,28 @@ from hierarchically_pruned_sparse_b200 import workloads as W
 # Attention tolerance for bf16 inputs (stated with the method's targets):
 # max |gpu - oracle| <= 2e-2 and mean <= 5e-3. For fp32 inputs the only error
 # sources are fp32 accumulation and exp2f over <= 10^6 keys: 2e-4 / 2e-5.
-TOL = {"bf16": (2e-2, 5e-3), "f32": (2e-4, 2e-5)}
+# fp8 e5m2 K/V widen exactly and the outputs are bf16: the bf16 tolerance.
+TOL = {"bf16": (2e-2, 5e-3), "f32": (2e-4, 2e-5), "e5m2": (2e-2, 5e-3)}
 NEAR_TIE = 1e-3          # rows whose oracle cut gap is below this may differ
 NEAR_TIE_MAX_FRAC = 0.005
 
 
 def torch_inputs(x: dict, w: W.Workload, step: int = 0):
+    """Device q, k, v of a workload (e5m2: bf16 q, uint8 code k and v)."""
     import torch
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    kt = torch.uint8 if w.dtype == "e5m2" else dt
     q = torch.from_numpy(np.ascontiguousarray(x["q"][step])).to("cuda").to(dt).contiguous()
-    k = torch.from_numpy(x["k"]).to("cuda").to(dt).contiguous()
-    v = torch.from_numpy(x["v"]).to("cuda").to(dt).contiguous()
+    k = torch.from_numpy(x["k"]).to("cuda").to(kt).contiguous()
+    v = torch.from_numpy(x["v"]).to("cuda").to(kt).contiguous()
     return q, k, v
+
+
+def oracle_kv(x: dict, w: W.Workload):
+    """float32 k, v for the oracle: the oracle decodes e5m2 codes itself."""
+    if w.dtype == "e5m2":
+        return oracle.decode_e5m2(x["k"]), oracle.decode_e5m2(x["v"])
+    return x["k"], x["v"]
 
 
 def shapes(w: W.Workload, step: int = 0):
@@ -35,7 +45,8 @@ def shapes(w: W.Workload, step: int = 0):
                   topk=w.topk, sink=w.sink, window=w.window, mask_len=w.seq_len,
                   kv_capacity=w.capacity)
     osh = oracle.shape(head_dim=w.head_dim, **common)
-    bkw = dict(dtype=hb.HIPS_BF16 if w.dtype == "bf16" else hb.HIPS_F32, **common)
+    code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
+    bkw = dict(dtype=code, **common)
     return osh, bkw
 
 

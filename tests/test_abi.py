@@ -134,3 +134,25 @@ def test_prefill_shapes_plan():
     p = hb.params(batch=1, n_qheads=32, n_kvheads=8, seq_len=32768, q_len=32768, q_pos0=0,
                   dtype=hb.HIPS_BF16, block_q=64, block_k=2, topk=2048, sink=128, window=1024)
     assert hb.idx_row_stride(p) == 1 + 1024 + 64 + 544 + 1
+
+
+def test_e5m2_kv_plans_decode_and_rejects_other_shapes():
+    f = 1 << 20
+    p = _decode_params(dtype=hb.HIPS_BF16_E5M2)
+    for op in (hb.OP_MASK, hb.OP_SPARSE, hb.OP_DENSE, hb.OP_MASK_SPARSE):
+        assert hb.workspace_size(p, op) >= 256, op
+    assert hb.mask_ptr(f, f, p, f) == hb.HIPS_ERR_WORKSPACE  # valid up to the missing workspace
+    # more than 16 rows per mask (one MMA column block) has no e5m2 mask kernel
+    wide = _decode_params(dtype=hb.HIPS_BF16_E5M2, n_qheads=64, n_kvheads=2)
+    assert hb.workspace_size(wide, hb.OP_MASK) == 0
+    assert hb.mask_ptr(f, f, wide, f) == hb.HIPS_ERR_UNSUPPORTED
+    # prefill query blocks: neither the mask nor the attention has an e5m2 kernel
+    pre = hb.params(batch=1, n_qheads=32, n_kvheads=8, seq_len=32768, q_len=32768, q_pos0=0,
+                    dtype=hb.HIPS_BF16_E5M2, block_q=64, block_k=2, topk=2048, sink=128,
+                    window=1024)
+    assert hb.workspace_size(pre, hb.OP_MASK) == 0
+    assert hb.workspace_size(pre, hb.OP_SPARSE) == 0
+    # more than 1024 chunks per mask does not fit beside the staging tiles
+    big = _decode_params(dtype=hb.HIPS_BF16_E5M2, topk=4096)
+    assert hb.workspace_size(big, hb.OP_MASK) == 0
+    assert hb.workspace_size(_decode_params(topk=4096), hb.OP_MASK) >= 256  # bf16 has a kernel

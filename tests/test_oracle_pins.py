@@ -18,6 +18,7 @@ import numpy as np
 import pytest
 
 import oracle
+from hierarchically_pruned_sparse_b200 import workloads as W
 from tests import brute_force as bf
 
 
@@ -427,3 +428,49 @@ def test_per_head_attention_reads_each_heads_own_row():
         np.testing.assert_allclose(out[0, h], ref[0], atol=2e-6, rtol=0)
     # the two query heads of a group do pick different blocks here
     assert not np.array_equal(idx[0], idx[1]) or not np.array_equal(idx[2], idx[3])
+
+
+# ---- fp8 e5m2 codes (the KV cache type of the SGLang integration's serving
+# commands, "[Feature] Support Efficient Sparse HiP Attention (InfiniteHiP)";
+# values per the OCP 8-bit floating-point format, E5M2)
+
+
+def test_e5m2_codes_are_the_upper_byte_of_binary16():
+    # numpy's IEEE binary16 conversion is an independent statement of the
+    # format: an e5m2 code c is the binary16 encoding c << 8
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.decode_e5m2(codes)
+    ref = (codes.astype(np.uint16) << np.uint16(8)).view(np.float16).astype(np.float32)
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x80, -0.0),
+    (0x3C, 1.0), (0xBC, -1.0), (0x40, 2.0), (0x3D, 1.25), (0x3F, 1.75),
+    (0x04, 2.0 ** -14),              # smallest normal
+    (0x01, 2.0 ** -16),              # smallest subnormal: 1/4 * 2^-14
+    (0x03, 3.0 * 2.0 ** -16),
+    (0x7B, 57344.0),                 # largest finite: 1.75 * 2^15
+    (0x7C, np.inf), (0xFC, -np.inf),
+])
+def test_e5m2_closed_form_values(code, value):
+    got = oracle.decode_e5m2(np.array([code], dtype=np.uint8))[0]
+    assert got == value and np.signbit(got) == np.signbit(value)
+
+
+def test_e5m2_nan_codes():
+    got = oracle.decode_e5m2(np.array([0x7D, 0x7E, 0x7F, 0xFD, 0xFE, 0xFF], dtype=np.uint8))
+    assert np.all(np.isnan(got))
+
+
+def test_e5m2_generator_codes_round_to_nearest():
+    # the generator's codes decode to a value nearest the drawn one among
+    # the finite e5m2 values (checked by brute force over the code table)
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(4000) * np.float32(3.0)).astype(np.float32)
+    codes = W.e5m2_codes(x)
+    table = oracle.decode_e5m2(np.arange(256, dtype=np.uint8)).astype(np.float64)
+    finite = np.isfinite(table)
+    got = oracle.decode_e5m2(codes).astype(np.float64)
+    best = np.min(np.abs(table[finite][None, :] - x[:, None].astype(np.float64)), axis=1)
+    assert np.all(np.abs(got - x) <= best * (1 + 1e-12))
