@@ -8,6 +8,7 @@ import pytest
 
 from hierarchically_pruned_sparse_b200 import binding as hb
 from hierarchically_pruned_sparse_b200 import build as hbuild
+from hierarchically_pruned_sparse_b200 import workloads as W
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -156,3 +157,35 @@ def test_e5m2_kv_plans_decode_and_rejects_other_shapes():
     big = _decode_params(dtype=hb.HIPS_BF16_E5M2, topk=4096)
     assert hb.workspace_size(big, hb.OP_MASK) == 0
     assert hb.workspace_size(_decode_params(topk=4096), hb.OP_MASK) >= 256  # bf16 has a kernel
+
+
+@pytest.mark.parametrize("name", sorted(W.WORKLOADS))
+def test_every_workload_plans_every_op(name):
+    # each benchmarked workload (and its mask reuse steps) has a kernel plan
+    # for the mask, the sparse and dense attention and the one-call step
+    w = W.WORKLOADS[name]
+    code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
+    T = w.seq_len
+    q_len = 1 if w.kind == "decode" else T
+    p = hb.params(batch=w.batch, n_qheads=w.n_qheads, n_kvheads=w.n_kvheads, seq_len=T,
+                  q_len=q_len, q_pos0=T - q_len, dtype=code, block_q=w.block_q,
+                  block_k=w.block_k, topk=w.topk, sink=w.sink, window=w.window,
+                  kv_capacity=w.capacity)
+    for op in (hb.OP_MASK, hb.OP_SPARSE, hb.OP_DENSE, hb.OP_MASK_SPARSE):
+        assert hb.workspace_size(p, op) >= 256, (name, op)
+    if w.refresh > 1:  # a later step attends the keys appended since the refresh
+        later = hb.params(batch=w.batch, n_qheads=w.n_qheads, n_kvheads=w.n_kvheads,
+                          seq_len=T + w.refresh - 1, q_len=1, q_pos0=T + w.refresh - 2,
+                          dtype=code, block_q=w.block_q, block_k=w.block_k, topk=w.topk,
+                          sink=w.sink, window=w.window, mask_len=T, kv_capacity=w.capacity)
+        assert hb.workspace_size(later, hb.OP_SPARSE) >= 256
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_head_masks_plan_decode_and_prefill(flags):
+    for q_len, bq in ((1, 1), (4096, 64)):
+        p = hb.params(batch=1, n_qheads=32, n_kvheads=8, seq_len=4096, q_len=q_len,
+                      q_pos0=4096 - q_len, dtype=hb.HIPS_BF16, block_q=bq, block_k=2,
+                      topk=512, sink=16, window=64, flags=flags)
+        assert hb.workspace_size(p, hb.OP_MASK) >= 256
+        assert hb.workspace_size(p, hb.OP_SPARSE) >= 256
