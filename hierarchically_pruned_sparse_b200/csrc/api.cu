@@ -79,11 +79,12 @@ struct MaskPlan {
   hips::MaskArgs a;
   int smem;
   size_t ws;
-  bool mma;  // tensor-core kernel (bf16) or CUDA-core kernel
+  bool mma;  // tensor-core kernel (bf16 or e5m2 keys) or CUDA-core kernel
   bool norms;  // key-block norm pre-pass into the workspace (many-row masks)
 };
 
-// Tensor-core mask plan: bf16, up to 256 query rows per mask, b_k <= 32.
+// Tensor-core mask plan: bf16 keys with up to 256 query rows per mask, or
+// e5m2 keys with up to 16 (one MMA column block); b_k <= 32.
 int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   hips::MaskArgs& a = plan->a;
   const int nc = hips::mask_mma_nc(a.rows_max);
