@@ -53,7 +53,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
@@ -64,6 +64,10 @@ def parse():
                     help="one mask per query head (head-reduce off) instead of per KV-head group")
     ap.add_argument("--two-calls", action="store_true",
                     help="decode: time hip_mask + hip_sparse_attn instead of hip_mask_sparse_attn")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="default run: leave out the nested prefill measurement")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="decode: leave out the dense-attention comparison")
     return ap.parse_args()
 
 
@@ -358,16 +362,6 @@ def reference_arm(args, w: W.Workload, world: int, rank: int):
     print(json.dumps(line), flush=True)
 
 
-def config_of(w: W.Workload, layers: int):
-    return {"workload": w.name, "kind": w.kind, "batch": w.batch, "seq_len": w.seq_len,
-            "n_qheads": w.n_qheads, "n_kvheads": w.n_kvheads, "head_dim": w.head_dim,
-            "topk": w.topk, "block_q": w.block_q, "block_k": w.block_k, "sink": w.sink,
-            "window": w.window, "parallelism": "replicas",
-            "masks": "per query head" if HEAD_MASKS else "per KV-head group",
-            "kv_cache": {"e5m2": "fp8 e5m2 (bf16 q and out)"}.get(w.dtype, w.dtype),
-            "l2": f"{layers} rotating layer buffers > L2 (no flush)" if layers else None}
-
-
 def _oracle_units(w: W.Workload, x: dict, sh, units: np.ndarray):
     """Oracle mask + attention of the given (sequence, KV head, query block) units."""
     import oracle
@@ -442,318 +436,561 @@ def traffic_from_profile(kernel: str, workload: str):
 # ---------------------------------------------------------------- our arm
 
 
-def ours(args, w: W.Workload, world: int, rank: int, local: int):
-    import torch
+def touched_bytes(w: W.Workload) -> int:
+    """Bytes one step of the workload reads (to size the rotating layer
+    buffers so that a layer's data has left L2 before it is used again):
+    prefill reads all of q, k and v; a decode refresh reads each round's
+    representative blocks and then the attended blocks."""
+    esz, kv_esz = elem_bytes(w)
+    wc = counting_view(w)
+    if w.kind == "prefill":
+        return (2 * w.batch * w.n_kvheads * w.capacity * kv_esz
+                + w.batch * w.n_qheads * w.q_len * esz) * w.head_dim
+    n = -(-w.seq_len // w.block_k)
+    n0 = min(w.topk // w.block_k, n)
+    rounds = max(0, math.ceil(math.log2(max(1, -(-n // n0)))))
+    units = wc.batch * wc.n_kvheads
+    attended = n0 + -(-w.sink // w.block_k) + (-(-w.window // w.block_k) + 1 if w.window else 0)
+    return units * (rounds * 2 * n0 + 2 * attended) * w.block_k * w.head_dim * kv_esz
 
-    from hierarchically_pruned_sparse_b200 import binding as hb
+
+def layer_count(w: W.Workload, layer_bytes: int, requested: int) -> int:
+    """Rotating layer buffers: enough that the bytes the steps between two uses
+    of a layer touch exceed 4x the L2, within 64 layers and 64 GB."""
+    if requested:
+        return requested
+    n = max(2, math.ceil(4 * L2_BYTES / max(1, touched_bytes(w))))
+    return max(2, min(n, 64, (64 << 30) // max(1, layer_bytes)))
+
+
+def config_of(w: W.Workload, layers: int):
+    cfg = {"workload": w.name, "kind": w.kind, "batch": w.batch, "seq_len": w.seq_len,
+           "n_qheads": w.n_qheads, "n_kvheads": w.n_kvheads, "head_dim": w.head_dim,
+           "topk": w.topk, "block_q": w.block_q, "block_k": w.block_k, "sink": w.sink,
+           "window": w.window, "parallelism": "replicas",
+           "masks": "per query head" if HEAD_MASKS else "per KV-head group",
+           "kv_cache": {"e5m2": "fp8 e5m2 (bf16 q and out)"}.get(w.dtype, w.dtype)}
+    if w.kind == "decode" and w.refresh > 1:
+        cfg["mask_refresh"] = w.refresh
+    if layers:
+        cfg["l2"] = (f"{layers} rotating layer buffers; the steps between two uses of a layer "
+                     f"touch {layers * touched_bytes(w) / L2_BYTES:.1f}x the L2 (no flush)")
+    return cfg
+
+
+def time_regions(replay, world: int, stream, dev, min_seconds: float = 1.0, max_regions: int = 5000):
+    """Device time of the timed region (K steps), repeated until at least
+    ``min_seconds`` of device time has passed: each repeat is bracketed by a
+    barrier and a device synchronisation on both sides and timed with CUDA
+    events on ``stream``; returns the per-repeat times (ms, max over ranks)."""
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def once():
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            replay()
+            end.record(stream)
+        end.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        return max_over_ranks(start.elapsed_time(end), world)
+
+    first = once()  # every rank sees the same maximum, so all agree on the count
+    n = int(min(max_regions, max(1, math.ceil(min_seconds * 1e3 / max(first, 1e-3)))))
+    return [first] + [once() for _ in range(n - 1)]
+
+
+class Layers:
+    """Device buffers of `layers` copies of a workload's layer: each layer's K
+    and V caches in one [2, ...] tensor (so that one copy appends a key row
+    and a value row), its own query per decode step, idx and output."""
+
+    def __init__(self, w: W.Workload, x: dict, layers: int, dev):
+        import torch
+        self.dt = torch.float32 if w.dtype == "f32" else torch.bfloat16  # q and out
+        self.kt = torch.uint8 if w.dtype == "e5m2" else self.dt          # k and v
+        k0 = torch.from_numpy(x["k"]).to(dev).to(self.kt).contiguous()
+        v0 = torch.from_numpy(x["v"]).to(dev).to(self.kt).contiguous()
+        self.kvs = [torch.stack([k0, v0]) for _ in range(layers)]
+        del k0, v0
+        self.ks = [kv[0] for kv in self.kvs]
+        self.vs = [kv[1] for kv in self.kvs]
+        steps = x["q"].shape[0]
+        qd = [torch.from_numpy(np.ascontiguousarray(x["q"][s])).to(dev).to(self.dt).contiguous()
+              for s in range(steps)]
+        self.qs = [[q.clone() for q in qd] for _ in range(layers)]  # [layer][decode step]
+        self.outs = [torch.empty_like(qd[0]) for _ in range(layers)]
+        self.n = layers
+
+
+def build_graph(stream, calls):
+    """A CUDA graph of the given calls, captured on ``stream``."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in calls:
+            c()
+    return g
+
+
+def ours(args, w: W.Workload, world: int, rank: int, local: int, nested: bool = False):
+    """Our arm on workload ``w``; returns the JSON line (printed by main)."""
+    import torch
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    x = W.make_inputs(w)
-    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16  # q and out
-    kt = torch.uint8 if w.dtype == "e5m2" else dt                # k and v
-    esz, kv_esz = elem_bytes(w)
-    prefill = w.kind == "prefill"
-    layer_bytes = 2 * x["k"].size * kv_esz + x["q"][0].size * esz
-    layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
-    layers = min(layers, 64)
-    k0 = torch.from_numpy(x["k"]).to(dev).to(kt).contiguous()
-    v0 = torch.from_numpy(x["v"]).to(dev).to(kt).contiguous()
-    q0 = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dev).to(dt).contiguous()
-    # each layer's K and V caches sit in one [2, ...] tensor, so that one copy
-    # appends a new key row and value row to both
-    kvs = [torch.stack([k0, v0]) for _ in range(layers)]
-    del k0, v0
-    ks = [kv[0] for kv in kvs]
-    vs = [kv[1] for kv in kvs]
-    qs = [q0.clone() for _ in range(layers)]
-    stream = torch.cuda.Stream(device=dev)
-    shp = layer_shape(w)
-    code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
-    sess = hb.Session(dtype=code,
-                      flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0,
-                      stream=stream, **shp)
-    idxs = [sess.new_idx() for _ in range(layers)]
-    outs = [torch.empty_like(q0) for _ in range(layers)]
+    if w.kind == "prefill":
+        return ours_prefill(args, w, world, rank, dev, nested)
+    return ours_decode(args, w, world, rank, dev)
 
-    # decode steps go through hip_mask_sparse_attn (a fresh mask and the
-    # attention over it); the library runs it as one launch for bf16 groups of
-    # at most 4 query rows, as the two kernels otherwise
-    fused = not prefill and not args.two_calls
-    wc = counting_view(w)
-    one_launch = fused and w.dtype != "f32" and wc.group * min(w.block_q, w.q_len) <= 4
 
-    def two_calls(l, q=None):
-        q = qs[l] if q is None else q
-        hb.hip_mask(q, ks[l], sess.p, idxs[l])
-        hb.hip_sparse_attn(q, ks[l], vs[l], idxs[l], sess.p, outs[l])
-
-    def step(l, q=None):
-        if fused:
-            hb.hip_mask_sparse_attn(qs[l] if q is None else q, ks[l], vs[l], sess.p, idxs[l],
-                                    outs[l])
-        else:
-            two_calls(l, q)
-
-    with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            step(i % layers)
-    stream.synchronize()
-    sess.check()
-    # one more mask call on a cleared status block counts the scored candidates
+def _scored_and_idx(hb, sess, lay, stream):
+    """Scored candidates of one mask call (status block counter) and its idx."""
     hb.workspace_init(sess.p)
-    with torch.cuda.stream(stream):
-        hb.hip_mask(qs[0], ks[0], sess.p, idxs[0])
+    with torch_stream(stream):
+        hb.hip_mask(lay.qs[0][0], lay.ks[0], sess.p, lay.idxs[0])
     stream.synchronize()
     base = sess.p.workspace - sess.workspace.data_ptr()
     scored = int(sess.workspace[base + 8: base + 16].cpu().numpy().view(np.uint64)[0])
     sess.check()
-    idx_host = idxs[0].cpu().numpy()
+    return scored, lay.idxs[0].cpu().numpy()
+
+
+def torch_stream(stream):
+    import torch
+    return torch.cuda.stream(stream)
+
+
+def ours_decode(args, w: W.Workload, world: int, rank: int, dev):
+    """Decode: a bench step is r_m decode steps of one layer (one mask refresh
+    through hip_mask_sparse_attn, then r_m - 1 steps of hip_sparse_attn that
+    reuse the mask while the cache grows by one key per step); with r_m = 1
+    every step refreshes. The calls run phase-major over the rotating layers
+    (decode step s of every layer, then step s + 1), as in a model."""
+    import torch
+
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    x = W.make_inputs(w)
+    esz, kv_esz = elem_bytes(w)
+    wc = counting_view(w)
+    rm = w.refresh
+    layer_bytes = 2 * x["k"].size * kv_esz + x["q"][0].size * esz
+    layers = layer_count(w, layer_bytes, args.layers)
+    lay = Layers(w, x, layers, dev)
+    stream = torch.cuda.Stream(device=dev)
+    shp = layer_shape(w)
+    code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
+    T = w.seq_len
+    # the workspace is sized at the longest cache of the reuse steps
+    shp.update(seq_len=T + rm - 1, q_pos0=T + rm - 2)
+    sess = hb.Session(dtype=code, flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0, stream=stream,
+                      mask_len=T, **shp)
+    sess.set(seq_len=T, q_pos0=T - 1)
+    lay.idxs = [sess.new_idx() for _ in range(layers)]
+    two = bool(args.two_calls)
+    one_launch = not two and w.dtype != "f32" and wc.group * min(w.block_q, w.q_len) <= 4
+
+    def call(l, s, q=None):
+        """Decode step s (0 = refresh) of layer l on query q (its own by default)."""
+        q = lay.qs[l][s] if q is None else q
+        sess.set(seq_len=T + s, mask_len=T, q_pos0=T + s - 1)
+        if s == 0 and not two:
+            hb.hip_mask_sparse_attn(q, lay.ks[l], lay.vs[l], sess.p, lay.idxs[l], lay.outs[l])
+        else:
+            if s == 0:
+                hb.hip_mask(q, lay.ks[l], sess.p, lay.idxs[l])
+            hb.hip_sparse_attn(q, lay.ks[l], lay.vs[l], lay.idxs[l], sess.p, lay.outs[l])
+
+    def cycle(nl):
+        """Calls of bench steps on layers [0, nl): phase-major."""
+        return [(l, s) for s in range(rm) for l in range(nl)]
+
+    with torch_stream(stream):
+        for i in range(max(args.warmup, 3)):  # untimed bench steps
+            for s in range(rm):
+                call(i % layers, s)
+    stream.synchronize()
+    sess.check()
+    sess.set(seq_len=T, mask_len=T, q_pos0=T - 1)
+    scored, idx_host = _scored_and_idx(hb, sess, lay, stream)
     mask_bytes = mask_algorithmic_bytes(wc, scored)
-    attn_bytes = attn_algorithmic_bytes(wc, idx_host, w.seq_len, w.seq_len)
-    mask_flops = mask_algorithmic_flops(wc, scored)
-    attn_flops = attn_algorithmic_flops(wc, idx_host) if prefill else 0
+    attn_bytes = [attn_algorithmic_bytes(wc, idx_host, T + s, T) for s in range(rm)]
+    step_bytes = mask_bytes + sum(attn_bytes)  # one bench step: r_m decode steps of a layer
 
-    # CUDA graphs of `layers` steps (and of the remainder of K); a copy of
-    # the full graph with event nodes around each kernel gives the kernel
-    # durations inside the timed region
-    def graph_with_events(ev, fused_step):
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            for l in range(layers):
-                ev[3 * l].record(stream)
-                if fused_step:
-                    hb.hip_mask_sparse_attn(qs[l], ks[l], vs[l], sess.p, idxs[l], outs[l])
-                    ev[3 * l + 1].record(stream)
-                else:
-                    hb.hip_mask(qs[l], ks[l], sess.p, idxs[l])
-                    ev[3 * l + 1].record(stream)
-                    hb.hip_sparse_attn(qs[l], ks[l], vs[l], idxs[l], sess.p, outs[l])
-                ev[3 * l + 2].record(stream)
-        return gr
-
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * layers)]
-    g_ev = graph_with_events(ev, fused)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for l in range(layers):
-            step(l)
     steps = max(1, args.steps)
     reps, rem = divmod(steps, layers)
-    g_rem = None
-    if rem:
-        g_rem = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_rem, stream=stream):
-            for l in range(rem):
-                step(l)
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            g.replay()
-            g_ev.replay()
-            if g_rem is not None:
-                g_rem.replay()
-    stream.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk, torch.cuda.stream(stream):
-        # graphs replay on the current stream: make it the stream the events use
-        start.record(stream)
-        # the last full replay carries the event nodes that time each kernel
-        for i in range(reps):
-            (g_ev if i == reps - 1 else g).replay()
+    g_full = build_graph(stream, [lambda l=l, s=s: call(l, s) for l, s in cycle(layers)])
+    g_rem = build_graph(stream, [lambda l=l, s=s: call(l, s) for l, s in cycle(rem)]) if rem else None
+
+    def replay():
+        for _ in range(reps):
+            g_full.replay()
         if g_rem is not None:
             g_rem.replay()
-        end.record(stream)
-        end.synchronize()
-    torch.cuda.synchronize(dev)
-    barrier(world)
+
+    with torch_stream(stream):
+        for _ in range(2):
+            replay()
+    stream.synchronize()
+    with ClockSampler(int(dev.index or 0)) as clk:
+        regions = time_regions(replay, world, stream, dev)
     sess.check()
-    total_ms = start.elapsed_time(end)
-    mask_ms = np.mean([ev[3 * l].elapsed_time(ev[3 * l + 1]) for l in range(layers)])
-    attn_ms = np.mean([ev[3 * l + 1].elapsed_time(ev[3 * l + 2]) for l in range(layers)])
-    total_ms = max_over_ranks(total_ms, world)
-    us_layer = whole_job_us_per_layer(total_ms, steps, world)
+    region_ms = float(np.median(regions))
+    step_us = region_ms * 1e3 / steps                      # one bench step (r_m decode steps)
+    us_layer = whole_job_us_per_layer(region_ms, steps * rm, world)  # per layer decode step
+
+    # split of a bench step by kernel: CUDA event nodes around each call of
+    # the first layer, in graph replays outside the timed region (the nodes
+    # add a little time of their own; the shares are what is reported)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * rm)]
+
+    def evcall(s):
+        def f():
+            ev[3 * s].record(stream)
+            sess.set(seq_len=T + s, mask_len=T, q_pos0=T + s - 1)
+            q = lay.qs[0][s]
+            if s == 0 and not two:
+                hb.hip_mask_sparse_attn(q, lay.ks[0], lay.vs[0], sess.p, lay.idxs[0], lay.outs[0])
+                ev[1].record(stream)
+            else:
+                if s == 0:
+                    hb.hip_mask(q, lay.ks[0], sess.p, lay.idxs[0])
+                ev[3 * s + 1].record(stream)
+                hb.hip_sparse_attn(q, lay.ks[0], lay.vs[0], lay.idxs[0], sess.p, lay.outs[0])
+            ev[3 * s + 2].record(stream)
+        return f
+
+    calls_ev = []
+    for l, s in cycle(layers):
+        calls_ev.append(evcall(s) if l == 0 else (lambda l=l, s=s: call(l, s)))
+    g_ev = build_graph(stream, calls_ev)
+    mask_ev, attn_ev = [], [[] for _ in range(rm)]
+    with torch_stream(stream):
+        for _ in range(max(3, min(30, 3000 // max(1, layers * rm)))):
+            g_ev.replay()
+            stream.synchronize()
+            mask_ev.append(ev[0].elapsed_time(ev[1]))
+            for s in range(rm):
+                attn_ev[s].append(ev[3 * s + 1].elapsed_time(ev[3 * s + 2]))
+    sess.check()
+    m_ev = float(np.median(mask_ev)) * 1e3
+    a_ev = [float(np.median(a)) * 1e3 for a in attn_ev]
+    # scale the event-node intervals to the measured step so that the
+    # per-kernel times add up to it (they cannot exceed the step)
+    ev_total = m_ev + sum(a_ev)
+    scale = step_us / ev_total if ev_total > 0 else 1.0
+    refresh_us = (m_ev + a_ev[0]) * scale
+    mask_us = m_ev * scale
+    attn0_us = a_ev[0] * scale
+    reuse_us = [a * scale for a in a_ev[1:]]
+
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
-    tensor_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-    mask_gbs = mask_bytes / (mask_ms * 1e-3) / 1e9
-    attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
-    step_gbs = (mask_bytes + attn_bytes) / (total_ms * 1e-3 / (steps)) / 1e9
-    mask_tf = mask_flops / (mask_ms * 1e-3) / 1e12
-    attn_tf = attn_flops / (attn_ms * 1e-3) / 1e12
-    step_tf = (mask_flops + attn_flops) / (total_ms * 1e-3 / steps) / 1e12
-    # hip_mask + hip_sparse_attn (their split merge is fused), or one launch
-    launches_per_step = 1 if one_launch else 2
-    if w.dtype == "bf16" and wc.group * min(w.block_q, w.q_len) > 32:
-        launches_per_step += 1  # the key-block norm pre-pass of a many-row mask
-    two_call = None
-    if fused:
-        # the same step as the two separate calls, for comparison (not timed above)
-        ev2 = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * layers)]
-        g3 = graph_with_events(ev2, False)
-        with torch.cuda.stream(stream):
-            for _ in range(max(3, min(50, reps))):
-                g3.replay()
+    if one_launch:
+        # the refresh is one kernel: mask and attention bytes over its time
+        dom_bytes, dom_us = mask_bytes + attn_bytes[0], refresh_us
+        dom_kernel = "mask_mma_kernel (mask + attention)"
+        traffic = traffic_from_profile("mask_mma_kernel+attn", w.name)
+    else:
+        dom_bytes, dom_us = mask_bytes, mask_us
+        dom_kernel = "mask_mma_kernel" if w.dtype != "f32" else "mask_fma_kernel"
+        traffic = traffic_from_profile(dom_kernel, w.name)
+    dom_gbs = dom_bytes / (dom_us * 1e-6) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom_kernel, "achieved": dom_gbs, "peak": hbm,
+                "peak_kind": f"{pk_kind} HBM copy", "unit": "GB/s", "frac": dom_gbs / hbm,
+                "traffic": traffic, "algorithmic_bytes": dom_bytes,
+                "time_us": dom_us,
+                "how": ("the refresh step's share of the median timed step (event-node "
+                        "split), algorithmic bytes over it" if rm > 1 or not one_launch else
+                        "the step is this one launch: algorithmic bytes over the median step time")}
+    step_gbs = step_bytes / (step_us * 1e-6) / 1e9
+    launches_refresh = 1 if one_launch else 2
+    launches_per_step = launches_refresh + (rm - 1)
+
+    kern = {"how": "median timed step split by CUDA event-node intervals of one layer "
+                   "(replays outside the timed region), scaled to the step",
+            "step_call": "hip_mask + hip_sparse_attn" if two else "hip_mask_sparse_attn",
+            "one_launch": one_launch, "scored_candidates": scored,
+            "mask_bytes": mask_bytes, "attn_bytes": attn_bytes[0]}
+    if one_launch:
+        kern["refresh_us"] = refresh_us
+    else:
+        kern.update(mask_us=mask_us, attn_us=attn0_us)
+    if rm > 1:
+        kern["refresh_us"] = refresh_us
+        kern["reuse_us_mean"] = float(np.mean(reuse_us))
+        kern["reuse_bytes_mean"] = float(np.mean(attn_bytes[1:]))
+        kern["reuse_gbs"] = kern["reuse_bytes_mean"] / (kern["reuse_us_mean"] * 1e-6) / 1e9
+    kern["event_node_us"] = {"mask_or_fused": m_ev, "attn": a_ev}
+
+    # the library's dense decode kernel on the same layers (comparison only)
+    dense = None
+    if not args.no_dense:
+        sess.set(seq_len=T, mask_len=T, q_pos0=T - 1)
+        gd = build_graph(stream, [lambda l=l: hb.hip_dense_attn(lay.qs[l][0], lay.ks[l], lay.vs[l],
+                                                                 sess.p, lay.outs[l])
+                                  for l in range(layers)])
+        with torch_stream(stream):
+            gd.replay()
         stream.synchronize()
+        dts = time_regions(lambda: gd.replay(), world, stream, dev, min_seconds=0.3)
         sess.check()
-        m2 = np.mean([ev2[3 * l].elapsed_time(ev2[3 * l + 1]) for l in range(layers)])
-        a2 = np.mean([ev2[3 * l + 1].elapsed_time(ev2[3 * l + 2]) for l in range(layers)])
-        two_call = {"mask_us": m2 * 1e3, "attn_us": a2 * 1e3, "step_us": (m2 + a2) * 1e3,
-                    "how": "hip_mask + hip_sparse_attn, CUDA event nodes, last of up to 50 replays"}
-        del g3
+        d_us = float(np.median(dts)) * 1e3 / layers
+        d_bytes = (wc.batch * w.n_kvheads * T * 2 * w.head_dim * kv_esz
+                   + 2 * w.batch * w.n_qheads * w.head_dim * esz)
+        dense = {"kernel": "attn_fma_kernel (dense)", "us_per_layer": d_us,
+                 "bytes": d_bytes, "gbs": d_bytes / (d_us * 1e-6) / 1e9,
+                 "frac": d_bytes / (d_us * 1e-6) / 1e9 / hbm,
+                 "speedup_of_sparse": d_us / us_layer}
+        del gd
 
-    # e2e: per step, one H2D from pinned host memory of the step's query and
-    # its new key and value rows (packed), one copy that appends the rows to the
-    # caches, the C-ABI call(s) on the query in the staging buffer, and D2H of
-    # the output; captured as a graph
-    e2e = None
-    if not args.no_e2e and not prefill:
-        # q (as bf16/f32 bytes) then the new key and value rows (native bytes)
-        q_host = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dt).contiguous().view(torch.uint8)
-        rows = torch.from_numpy(np.ascontiguousarray(
-            np.stack([x["k"][:, :, w.seq_len - 1], x["v"][:, :, w.seq_len - 1]])))
-        rows = rows.to(kt).contiguous()
-        rb = rows.view(torch.uint8).reshape(-1)
-        packed = torch.cat([q_host.reshape(-1), rb])
-        hstage = [packed.clone().pin_memory() for _ in range(layers)]
-        dstage = [torch.empty(packed.numel(), dtype=torch.uint8, device=dev) for _ in range(layers)]
-        qv = [d[:q_host.numel()].view(dt).view(q0.shape) for d in dstage]
-        kvrow = [d[q_host.numel():].view(kt).view(rows.shape) for d in dstage]
-        hout = [torch.empty(q0.shape, dtype=dt).pin_memory() for _ in range(layers)]
-
-        def e2e_step(l):
-            dstage[l].copy_(hstage[l], non_blocking=True)
-            kvs[l][:, :, :, w.seq_len - 1].copy_(kvrow[l])
-            step(l, qv[l])
-            hout[l].copy_(outs[l], non_blocking=True)
-
-        g2 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g2, stream=stream):
-            for l in range(layers):
-                e2e_step(l)
-        g2_rem = None
-        if rem:
-            g2_rem = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g2_rem, stream=stream):
-                for l in range(rem):
-                    e2e_step(l)
-        with torch.cuda.stream(stream):
-            g2.replay()
-        stream.synchronize()
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        with torch.cuda.stream(stream):
-            s2.record(stream)
-            for _ in range(reps):
-                g2.replay()
-            if g2_rem is not None:
-                g2_rem.replay()
-            e2.record(stream)
-        e2.synchronize()
-        barrier(world)
-        e2e_ms = max_over_ranks(s2.elapsed_time(e2), world)
-        h2d = packed.numel()
-        e2e = {"value": whole_job_us_per_layer(e2e_ms, steps, world), "unit": "us/layer",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(q0.numel() * esz),
-               "how": "CUDA graph per step: one H2D (pinned) of q and the new k/v rows, "
-                      "their append to the caches, "
-                      + ("hip_mask_sparse_attn" if fused else "hip_mask + hip_sparse_attn")
-                      + ", D2H of out"}
-        sess.check()
-
-    if not args.no_e2e and prefill:
-        hq = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(dt).pin_memory()
-        hk = torch.from_numpy(x["k"]).to(dt).pin_memory()
-        hv = torch.from_numpy(x["v"]).to(dt).pin_memory()
-        hout = torch.empty(q0.shape, dtype=dt).pin_memory()
-        n_e2e = max(1, min(steps, 20))
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        with torch.cuda.stream(stream):
-            s2.record(stream)
-            for i in range(n_e2e):
-                l = i % layers
-                qs[l].copy_(hq, non_blocking=True)
-                ks[l].copy_(hk, non_blocking=True)
-                vs[l].copy_(hv, non_blocking=True)
-                step(l)
-                hout.copy_(outs[l], non_blocking=True)
-            e2.record(stream)
-        e2.synchronize()
-        barrier(world)
-        e2e_ms = max_over_ranks(s2.elapsed_time(e2), world)
-        fl = (mask_flops + attn_flops) * n_e2e * world
-        e2e = {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": int((hq.numel() + hk.numel() + hv.numel()) * esz),
-               "d2h_bytes_per_step": int(q0.numel() * esz), "steps": n_e2e,
-               "how": "per step: H2D of q, k, v (pinned), hip_mask, hip_sparse_attn, D2H of out"}
-        sess.check()
-
+    e2e = None if args.no_e2e else decode_e2e(args, w, x, lay, sess, call, cycle, steps, layers,
+                                               world, stream, dev, esz)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, x)
 
-    mask_kernel = "mask_mma_kernel" if w.dtype != "f32" else "mask_fma_kernel"
-    attn_kernel = "attn_mma_kernel" if prefill else "attn_fma_kernel"
-    if prefill:
-        dom_attn = attn_ms >= mask_ms
-        dom_tf = attn_tf if dom_attn else mask_tf
-        roofline = {"bound": "tensor", "kernel": attn_kernel if dom_attn else mask_kernel,
-                    "achieved": dom_tf, "peak": tensor_peak, "peak_kind": f"{pk_kind} bf16 sustained",
-                    "unit": "TFLOP/s", "frac": dom_tf / tensor_peak,
-                    "traffic": traffic_from_profile(attn_kernel if dom_attn else mask_kernel, w.name),
-                    "algorithmic_flops": attn_flops if dom_attn else mask_flops}
-        value, unit, hib = step_tf, "TFLOP/s", True
-    else:
-        if one_launch:
-            # one kernel does the whole step: its bytes are the mask's and the attention's
-            fused_gbs = (mask_bytes + attn_bytes) / (mask_ms * 1e-3) / 1e9
-            roofline = {"bound": "hbm", "kernel": mask_kernel + " (mask + attention)",
-                        "achieved": fused_gbs, "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s",
-                        "frac": fused_gbs / hbm,
-                        "traffic": traffic_from_profile(mask_kernel + "+attn", w.name),
-                        "algorithmic_bytes": mask_bytes + attn_bytes}
-        else:
-            roofline = {"bound": "hbm", "kernel": mask_kernel, "achieved": mask_gbs,
-                        "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s", "frac": mask_gbs / hbm,
-                        "traffic": traffic_from_profile(mask_kernel, w.name),
-                        "algorithmic_bytes": mask_bytes}
-        value, unit, hib = us_layer, "us/layer", False
     line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
-        "steps": steps, "warmup": args.warmup, "ms_per_step": total_ms / steps,
-        "higher_is_better": hib, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+        "metric": METRIC, "value": us_layer, "unit": "us/layer", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": region_ms / steps,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if lay.dt == torch.bfloat16 else "f32",
         "data": "synthetic (seeded AR(1) keys/values, Gaussian queries, needle keys)",
         "config": config_of(w, layers),
         "roofline": roofline,
         "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": hbm, "unit": "GB/s",
-                          "frac": step_gbs / hbm, "algorithmic_bytes": mask_bytes + attn_bytes},
-        "kernels": {"how": "CUDA event nodes around each call, last full graph replay of the timed region",
-                    "step_call": "hip_mask_sparse_attn" if fused else "hip_mask + hip_sparse_attn",
-                    "one_launch": one_launch,
-                    "mask_kernel": mask_kernel, "attn_kernel": None if one_launch else attn_kernel,
-                    "mask_us": mask_ms * 1e3, "mask_bytes": mask_bytes, "mask_gbs": mask_gbs,
-                    "mask_tflops": mask_tf, "mask_flops": mask_flops, "scored_candidates": scored,
-                    "attn_us": attn_ms * 1e3, "attn_bytes": attn_bytes, "attn_gbs": attn_gbs,
-                    "attn_tflops": attn_tf, "attn_flops": attn_flops},
+                          "frac": step_gbs / hbm, "algorithmic_bytes": step_bytes},
+        "kernels": kern,
+        "timing": {"regions": len(regions), "region_ms_median": region_ms,
+                   "region_ms_min": float(np.min(regions)), "region_ms_max": float(np.max(regions)),
+                   "decode_steps_per_bench_step": rm},
         "gpu_launches": launches_per_step * steps,
         "clocks": clk.summary(),
     }
-    if two_call:
-        line["kernels"]["two_calls"] = two_call
-    if prefill:
-        line["step_tflops"] = step_tf
-        line["us_per_layer"] = us_layer
+    if dense:
+        line["dense"] = dense
     if e2e:
         line["e2e"] = e2e
     if cpu:
         line["cpu_baseline"] = cpu
-    del g, g_ev, g_rem
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    return line
+
+
+def decode_e2e(args, w, x, lay, sess, call, cycle, steps, layers, world, stream, dev, esz):
+    """End to end through the C ABI: per decode call one H2D (pinned host) of
+    the call's query and new key and value rows, packed, on a copy stream;
+    one copy appends the rows to the caches; the call itself on the query in
+    the staging buffer; and a D2H of the output. The uploads of later calls
+    overlap the kernels of earlier ones (they do not depend on them)."""
+    import torch
+    dt, kt = lay.dt, lay.kt
+    T = w.seq_len
+    rm = w.refresh
+    copy_stream = torch.cuda.Stream(device=dev)
+    n_calls = layers * rm
+    q_host = [torch.from_numpy(np.ascontiguousarray(x["q"][s])).to(dt).contiguous().view(torch.uint8)
+              for s in range(rm)]
+    rows = [torch.from_numpy(np.ascontiguousarray(
+        np.stack([x["k"][:, :, T - 1 + s], x["v"][:, :, T - 1 + s]]))).to(kt).contiguous()
+        for s in range(rm)]
+    packed = [torch.cat([q_host[s].reshape(-1), rows[s].view(torch.uint8).reshape(-1)]) for s in range(rm)]
+    hstage = [[packed[s].clone().pin_memory() for s in range(rm)] for _ in range(layers)]
+    dstage = [[torch.empty(packed[s].numel(), dtype=torch.uint8, device=dev) for s in range(rm)]
+              for _ in range(layers)]
+    nq = q_host[0].numel()
+    qv = [[d[:nq].view(dt).view(lay.qs[0][0].shape) for d in dl] for dl in dstage]
+    kvrow = [[d[nq:].view(kt).view(rows[0].shape) for d in dl] for dl in dstage]
+    hout = [[torch.empty(lay.outs[0].shape, dtype=dt).pin_memory() for _ in range(rm)]
+            for _ in range(layers)]
+    up = [torch.cuda.Event() for _ in range(n_calls)]
+
+    def e2e_calls(nl):
+        order = cycle(nl)
+
+        def run():
+            cur = torch.cuda.current_stream()
+            copy_stream.wait_stream(cur)
+            # uploads, in call order, on the copy stream
+            with torch.cuda.stream(copy_stream):
+                for i, (l, s) in enumerate(order):
+                    dstage[l][s].copy_(hstage[l][s], non_blocking=True)
+                    up[i].record(copy_stream)
+            for i, (l, s) in enumerate(order):
+                cur.wait_event(up[i])
+                lay.kvs[l][:, :, :, T - 1 + s].copy_(kvrow[l][s])
+                call(l, s, qv[l][s])
+                hout[l][s].copy_(lay.outs[l], non_blocking=True)
+            cur.wait_stream(copy_stream)
+        return run
+
+    reps, rem = divmod(steps, layers)
+    g2 = build_graph(stream, [e2e_calls(layers)])
+    g2_rem = build_graph(stream, [e2e_calls(rem)]) if rem else None
+
+    def replay():
+        for _ in range(reps):
+            g2.replay()
+        if g2_rem is not None:
+            g2_rem.replay()
+
+    with torch_stream(stream):
+        replay()
+    stream.synchronize()
+    regions = time_regions(replay, world, stream, dev, min_seconds=0.5)
+    sess.check()
+    e2e_ms = float(np.median(regions))
+    h2d = int(np.mean([p.numel() for p in packed]))
+    return {"value": whole_job_us_per_layer(e2e_ms, steps * rm, world), "unit": "us/layer",
+            "h2d_bytes_per_step": h2d * rm, "d2h_bytes_per_step": int(lay.outs[0].numel() * esz) * rm,
+            "regions": len(regions),
+            "how": "CUDA graph per group of steps: per decode call one H2D (pinned) of q and "
+                   "the new k/v rows on a copy stream (overlapping earlier calls' kernels), "
+                   "their append to the caches, the C-ABI call, D2H of out"}
+
+
+def ours_prefill(args, w: W.Workload, world: int, rank: int, dev, nested: bool):
+    """Prefill: a step is hip_mask (key-norm pre-pass and mask) and
+    hip_sparse_attn over the whole sequence, rotating over layer buffers."""
+    import torch
+
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    x = W.make_inputs(w)
+    esz, kv_esz = elem_bytes(w)
+    wc = counting_view(w)
+    layer_bytes = 2 * x["k"].size * kv_esz + x["q"][0].size * esz
+    layers = layer_count(w, layer_bytes, 0 if nested else args.layers)
+    lay = Layers(w, x, layers, dev)
+    stream = torch.cuda.Stream(device=dev)
+    code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
+    sess = hb.Session(dtype=code, flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0, stream=stream,
+                      **layer_shape(w))
+    lay.idxs = [sess.new_idx() for _ in range(layers)]
+
+    def call(l):
+        hb.hip_mask(lay.qs[l][0], lay.ks[l], sess.p, lay.idxs[l])
+        hb.hip_sparse_attn(lay.qs[l][0], lay.ks[l], lay.vs[l], lay.idxs[l], sess.p, lay.outs[l])
+
+    with torch_stream(stream):
+        for i in range(max(args.warmup, 3)):
+            call(i % layers)
+    stream.synchronize()
+    sess.check()
+    scored, idx_host = _scored_and_idx(hb, sess, lay, stream)
+    mask_flops = mask_algorithmic_flops(wc, scored)
+    attn_flops = attn_algorithmic_flops(wc, idx_host)
+    steps = max(1, args.steps)
+    reps, rem = divmod(steps, layers)
+    g_full = build_graph(stream, [lambda l=l: call(l) for l in range(layers)])
+    g_rem = build_graph(stream, [lambda l=l: call(l) for l in range(rem)]) if rem else None
+
+    def replay():
+        for _ in range(reps):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+
+    with torch_stream(stream):
+        replay()
+    stream.synchronize()
+    with ClockSampler(int(dev.index or 0)) as clk:
+        regions = time_regions(replay, world, stream, dev)
+    sess.check()
+    region_ms = float(np.median(regions))
+    step_ms = region_ms / steps
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+
+    def evcall():
+        ev[0].record(stream)
+        hb.hip_mask(lay.qs[0][0], lay.ks[0], sess.p, lay.idxs[0])
+        ev[1].record(stream)
+        hb.hip_sparse_attn(lay.qs[0][0], lay.ks[0], lay.vs[0], lay.idxs[0], sess.p, lay.outs[0])
+        ev[2].record(stream)
+
+    g_ev = build_graph(stream, [evcall] + [lambda l=l: call(l) for l in range(1, layers)])
+    m_ev, a_ev = [], []
+    with torch_stream(stream):
+        for _ in range(5):
+            g_ev.replay()
+            stream.synchronize()
+            m_ev.append(ev[0].elapsed_time(ev[1]))
+            a_ev.append(ev[1].elapsed_time(ev[2]))
+    sess.check()
+    m_ev, a_ev = float(np.median(m_ev)), float(np.median(a_ev))
+    scale = step_ms / (m_ev + a_ev)
+    mask_ms, attn_ms = m_ev * scale, a_ev * scale
+    pk, pk_kind = peaks()
+    burst = float(pk["bf16_tflops"])
+    sustained = float(pk.get("bf16_tflops_sustained", burst))
+    mask_tf = mask_flops / (mask_ms * 1e-3) / 1e12
+    attn_tf = attn_flops / (attn_ms * 1e-3) / 1e12
+    step_tf = (mask_flops + attn_flops) * world / (region_ms * 1e-3 / steps) / 1e12
+
+    def tensor_roof(kernel, tf, flops, ms):
+        return {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": burst,
+                "peak_kind": f"{pk_kind} bf16 burst (cuBLAS)", "unit": "TFLOP/s", "frac": tf / burst,
+                "frac_of_sustained": tf / sustained, "sustained_peak": sustained,
+                "traffic": traffic_from_profile(kernel, w.name), "algorithmic_flops": flops,
+                "time_ms": ms}
+
+    mask_kernel = "mask_mma_kernel"
+    roofline = (tensor_roof(mask_kernel, mask_tf, mask_flops, mask_ms) if mask_ms >= attn_ms
+                else tensor_roof("attn_mma_kernel", attn_tf, attn_flops, attn_ms))
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(np.ascontiguousarray(x["q"][0])).to(lay.dt).pin_memory()
+        hk = torch.from_numpy(x["k"]).to(lay.kt).pin_memory()
+        hv = torch.from_numpy(x["v"]).to(lay.kt).pin_memory()
+        hout = torch.empty(lay.outs[0].shape, dtype=lay.dt).pin_memory()
+        n_e2e = max(1, min(steps, 10))
+
+        def e2e_replay():
+            for i in range(n_e2e):
+                l = i % layers
+                lay.qs[l][0].copy_(hq, non_blocking=True)
+                lay.ks[l].copy_(hk, non_blocking=True)
+                lay.vs[l].copy_(hv, non_blocking=True)
+                call(l)
+                hout.copy_(lay.outs[l], non_blocking=True)
+
+        regions_e = time_regions(e2e_replay, world, stream, dev, min_seconds=0.0, max_regions=3)
+        sess.check()
+        e2e_ms = float(np.median(regions_e))
+        e2e = {"value": (mask_flops + attn_flops) * n_e2e * world / (e2e_ms * 1e-3) / 1e12,
+               "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int((hq.numel() * esz + (hk.numel() + hv.numel()) * kv_esz)),
+               "d2h_bytes_per_step": int(lay.outs[0].numel() * esz), "steps": n_e2e,
+               "how": "per step: H2D of q, k, v (pinned), hip_mask, hip_sparse_attn, D2H of out"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x)
+        if cpu:
+            cpu = dict(cpu, value_tflops=(mask_flops + attn_flops) / (cpu["value"] * 1e-6) / 1e12)
+    line = {
+        "metric": METRIC, "value": step_tf, "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if lay.dt == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded AR(1) queries, keys and values)",
+        "config": config_of(w, layers),
+        "roofline": roofline,
+        "attn_roofline": tensor_roof("attn_mma_kernel", attn_tf, attn_flops, attn_ms),
+        "mask_roofline": tensor_roof(mask_kernel, mask_tf, mask_flops, mask_ms),
+        "kernels": {"how": "median timed step split by CUDA event-node intervals (replays "
+                           "outside the timed region), scaled to the step",
+                    "mask_ms": mask_ms, "attn_ms": attn_ms, "mask_flops": mask_flops,
+                    "attn_flops": attn_flops, "scored_candidates": scored,
+                    "us_per_layer": step_ms * 1e3},
+        "timing": {"regions": len(regions), "region_ms_median": region_ms,
+                   "region_ms_min": float(np.min(regions)), "region_ms_max": float(np.max(regions))},
+        "gpu_launches": 3 * steps,  # key-norm pre-pass, mask, attention
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if cpu:
+        line["cpu_baseline"] = cpu
+    return line
 
 
 def main():
@@ -768,7 +1005,19 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        ours(args, w, world, rank, local)
+        line = ours(args, w, world, rank, local)
+        if (args.workload == DEFAULT_WORKLOAD and not args.no_prefill and not HEAD_MASKS
+                and not args.two_calls):
+            # the other half of the metric: prefill TFLOP/s, in the same line
+            pw = W.PREFILL_32K
+            pre = ours(args, pw, world, rank, local, nested=True)
+            line["prefill"] = {k: pre[k] for k in ("value", "unit", "ms_per_step", "config",
+                                                   "roofline", "attn_roofline", "mask_roofline",
+                                                   "kernels", "timing", "gpu_launches", "clocks",
+                                                   "e2e", "cpu_baseline") if k in pre}
+            line["gpu_launches_prefill"] = pre["gpu_launches"]
+        if rank == 0:
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist

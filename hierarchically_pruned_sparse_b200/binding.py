@@ -32,7 +32,7 @@ FLAG_HEAD_MASKS = 1  # one mask per query head (idx [B, Hq, n_qblocks, row_strid
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhip_sparse.so")
 EXPORTS = ("hip_idx_row_stride", "hip_workspace_size", "hip_workspace_init", "hip_check_status",
            "hip_mask", "hip_sparse_attn", "hip_mask_sparse_attn", "hip_dense_attn",
-           "hip_sparse_attn_noalloc", "hip_last_cuda_error",
+           "hip_sparse_attn_noalloc", "hip_noalloc_check_status", "hip_last_cuda_error",
            "hip_error_string")
 
 
@@ -91,6 +91,8 @@ def load() -> ctypes.CDLL:
     lib.hip_dense_attn.argtypes = [vp, vp, vp, P, vp]
     lib.hip_sparse_attn_noalloc.restype = ctypes.c_int
     lib.hip_sparse_attn_noalloc.argtypes = [vp, vp, vp, vp, P, vp]
+    lib.hip_noalloc_check_status.restype = ctypes.c_int
+    lib.hip_noalloc_check_status.argtypes = [vp]
     lib.hip_last_cuda_error.restype = ctypes.c_int
     lib.hip_last_cuda_error.argtypes = []
     lib.hip_error_string.restype = ctypes.c_char_p
@@ -201,6 +203,15 @@ def hip_sparse_attn_noalloc(q, k, v, idx, p: Params, out) -> None:
     split-K scratch is a fixed array inside the library (see the header)."""
     _check("hip_sparse_attn_noalloc",
            sparse_attn_noalloc_ptr(_dev(q), _dev(k), _dev(v), _dev(idx), p, _dev(out)))
+
+
+def noalloc_check_status(stream=None) -> None:
+    """Raise if the last hip_sparse_attn_noalloc call on this device gave up a
+    bounded wait (synchronises the stream; torch's current one by default)."""
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    _check("hip_noalloc_check_status", load().hip_noalloc_check_status(stream.cuda_stream or None))
 
 
 def hip_dense_attn(q, k, v, p: Params, out) -> None:

@@ -20,12 +20,9 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kPlanSMs = 148;         // B200 streaming multiprocessors
-// Head of every workspace: bytes [0, 256) hold the sticky status word, bytes
-// [256, 4096) one split-merge counter per (sequence, KV head, query block)
-// unit of a split attention call; both are zero between calls.
-constexpr size_t kStatusBytes = 4096;
-constexpr size_t kCounterOffset = 256;
-constexpr int64_t kMaxCounters = (kStatusBytes - kCounterOffset) / 4;
+using hips::kStatusBytes;             // workspace head layout (hips_kernels.h)
+using hips::kCounterOffset;
+using hips::kMaxCounters;
 constexpr int kMaxSmem = 227 * 1024;
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }

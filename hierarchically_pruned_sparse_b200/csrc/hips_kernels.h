@@ -10,6 +10,18 @@ namespace hips {
 
 struct Status;
 
+// Layout of the head of every workspace (and of the no-allocation entry
+// point's fixed scratch array): bytes [0, 256) hold the sticky status word,
+// bytes [256, 4096) one split-merge counter per (sequence, KV head, query
+// block) unit of a split attention call; both are zero between calls. The
+// split-K partials (or the key-norm table of a many-row mask) follow at 4096.
+constexpr size_t kStatusBytes = 4096;
+constexpr size_t kCounterOffset = 256;
+constexpr int64_t kMaxCounters = static_cast<int64_t>((kStatusBytes - kCounterOffset) / sizeof(unsigned int));
+static_assert(kCounterOffset >= 16, "the counters start after the status word");
+static_assert(kCounterOffset + kMaxCounters * sizeof(unsigned int) <= kStatusBytes,
+              "the counter area of kMaxCounters units lies inside the status block");
+
 struct MaskArgs {
   const void* q;
   const void* k;

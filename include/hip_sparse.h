@@ -186,17 +186,27 @@ HIPS_API int hip_dense_attn(const void* q, const void* k, const void* v, const h
  *    HIPS_OP_SPARSE) > HIPS_NOALLOC_SCRATCH_BYTES) return HIPS_ERR_TOO_LARGE
  *    before launching anything.
  *  - The first call on each device looks the array's device address up
- *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    (cudaGetSymbolAddress, with that device current) and caches it with the
+ *    device's context; the first call after a device reset looks it up
+ *    again. Make the first call on a device, and the first after a reset,
  *    before any stream capture.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents; each call clears the part that must start at zero. Calls that
  *    overlap on the GPU (different streams, or other host threads) race on
  *    it: serialise them.
- *  - Bounded-wait failures of this call are not reported through
- *    hip_check_status (it has no caller workspace). */
+ *  - A bounded device wait that gives up is recorded in the array's status
+ *    word, which the next call clears: read it with
+ *    hip_noalloc_check_status before the next call. */
 #define HIPS_NOALLOC_SCRATCH_BYTES (512u << 10)
 HIPS_API int hip_sparse_attn_noalloc(const void* q, const void* k, const void* v,
                                      const int32_t* idx, const hips_params* params, void* out);
+
+/* Status of the most recent hip_sparse_attn_noalloc call on the current
+ * device: synchronises `stream` (a cudaStream_t), reads the status word of
+ * the library's fixed array and clears it. Returns HIPS_OK, or
+ * HIPS_ERR_TIMEOUT if that call's kernel gave up a bounded wait (its output
+ * is then undefined), or HIPS_ERR_CUDA. Allocates nothing either. */
+HIPS_API int hip_noalloc_check_status(void* stream);
 
 /* cudaError_t of the last failed launch on this thread (0 if none). */
 HIPS_API int hip_last_cuda_error(void);

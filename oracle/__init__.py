@@ -74,6 +74,9 @@ def _load():
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_mask.restype = ctypes.c_int
     lib.oracle_mask.argtypes = [f32p, f32p, P(Shape), i64p, ctypes.c_int64, i32p, f64p, i32p, i64p]
+    lib.oracle_block_scores.restype = ctypes.c_int
+    lib.oracle_block_scores.argtypes = [f32p, f32p, P(Shape), ctypes.c_int64, i64p, ctypes.c_int64,
+                                        f32p]
     lib.oracle_decode_e5m2.restype = None
     lib.oracle_decode_e5m2.argtypes = [P(ctypes.c_uint8), ctypes.c_int64, f32p]
     lib.oracle_attention.restype = ctypes.c_int
@@ -157,6 +160,22 @@ def mask(q, k, sh: Shape, units=None, with_scored=False):
     if with_scored:
         return idx, gap, rounds, scored
     return idx, gap, rounds
+
+
+def block_scores(q, k, sh: Shape, unit: int, blocks) -> np.ndarray:
+    """float32 scores (step 3 of the rounds: max over the unit's query rows and
+    the block's visible keys of the canonical dot) of the given key blocks of
+    one mask row; -inf outside the unit's block range."""
+    lib = _load()
+    q, k = _f32(q), _f32(k)
+    b = np.ascontiguousarray(blocks, dtype=np.int64)
+    out = np.empty(b.size, dtype=np.float32)
+    st = lib.oracle_block_scores(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                 ctypes.byref(sh), int(unit), _ptr(b, ctypes.c_int64), b.size,
+                                 _ptr(out, ctypes.c_float))
+    if st != 0:
+        raise RuntimeError(f"oracle_block_scores failed ({st})")
+    return out
 
 
 def attention(q, k, v, idx, sh: Shape, rows=None) -> np.ndarray:

@@ -161,25 +161,85 @@ static int cand_order(const void* pa, const void* pb) {
   return (a->s > b->s) - (a->s < b->s);
 }
 
+/* The query rows and the key range of one mask row (unit). */
+typedef struct {
+  int64_t b, g, h0, i0, i1, q_first, q_last, Tc, N, n0;
+  int Gm;
+} unit_rows;
+
+static int unit_setup(const oracle_shape* sh, int64_t unit, unit_rows* u) {
+  const int G = sh->n_qheads / sh->n_kvheads;
+  const int64_t nqb = oracle_num_qblocks(sh), bk = sh->block_k;
+  /* the mask's heads: G query heads sharing KV head g, or one query head */
+  const int64_t mh = sh->per_head ? sh->n_qheads : sh->n_kvheads;
+  const int64_t total = (int64_t)sh->batch * mh * nqb;
+  if (unit < 0 || unit >= total) return OR_BAD;
+  const int64_t qb = unit % nqb, hm = (unit / nqb) % mh;
+  u->b = unit / (nqb * mh);
+  u->g = sh->per_head ? hm / G : hm;       /* KV head */
+  u->Gm = sh->per_head ? 1 : G;            /* query heads of the mask */
+  u->h0 = sh->per_head ? hm : hm * G;      /* first of them */
+  u->i0 = qb * sh->block_q;
+  u->i1 = min64(u->i0 + sh->block_q, sh->q_len);
+  u->q_first = sh->q_pos0 + u->i0;
+  u->q_last = sh->q_pos0 + u->i1 - 1;
+  u->Tc = min64(u->q_last + 1, sh->seq_len);
+  u->N = cdiv64(u->Tc, bk);
+  u->n0 = min64(sh->topk / bk, u->N);
+  return OR_OK;
+}
+
+/* [RsGC] step 3: the score of key block `rep` for the unit's query rows: the
+ * max over the rows and the block's keys j < Tc, j <= p (causal) of the
+ * canonical dot q.k; -inf when no row sees a key of the block. */
+static float block_score(const float* q, const float* k, const oracle_shape* sh,
+                         const unit_rows* u, int64_t rep) {
+  const int d = sh->head_dim;
+  const int64_t bk = sh->block_k;
+  float best = -INFINITY;
+  for (int h = 0; h < u->Gm; ++h) {
+    const int64_t qh = u->h0 + h;
+    for (int64_t i = u->i0; i < u->i1; ++i) {
+      const int64_t p = sh->q_pos0 + i;
+      const float* qr = q + (((u->b * sh->n_qheads + qh) * sh->q_len + i) * d);
+      for (int64_t j = rep * bk; j < min64(rep * bk + bk, u->Tc); ++j) {
+        if (j > p) continue;
+        const float* kj = k + (((u->b * sh->n_kvheads + u->g) * sh->kv_capacity + j) * d);
+        float sc = oracle_canonical_dot(qr, kj, d);
+        if (sc > best) best = sc;
+      }
+    }
+  }
+  return best;
+}
+
+/*
+ * Scores of explicit key blocks for one unit (the step-3 score above), so
+ * that a test can replay the rounds along another selection path: out[i] is
+ * the score of blocks[i] (-inf for a block outside [0, N)).
+ */
+int oracle_block_scores(const float* q, const float* k, const oracle_shape* sh, int64_t unit,
+                        const int64_t* blocks, int64_t n, float* out) {
+  if (!q || !k || !out || (n > 0 && !blocks) || !shape_ok(sh)) return OR_BAD;
+  unit_rows u;
+  if (unit_setup(sh, unit, &u) != OR_OK) return OR_BAD;
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = (blocks[i] >= 0 && blocks[i] < u.N) ? block_score(q, k, sh, &u, blocks[i]) : -INFINITY;
+  return OR_OK;
+}
+
 /*
  * One mask row: sequence b, KV head g, query block qb ([RsGC] steps 1-4,
  * then the sink/window union of [Summary] and the idx+nnz row of [NLBm] W2).
  */
 static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int64_t unit,
                      int32_t* row, double* gap_out, int32_t* rounds_out, int64_t* scored_out) {
-  const int d = sh->head_dim, G = sh->n_qheads / sh->n_kvheads;
-  const int64_t nqb = oracle_num_qblocks(sh), bk = sh->block_k;
-  /* the mask's heads: G query heads sharing KV head g, or one query head */
-  const int64_t mh = sh->per_head ? sh->n_qheads : sh->n_kvheads;
-  const int64_t qb = unit % nqb, hm = (unit / nqb) % mh, b = unit / (nqb * mh);
-  const int64_t g = sh->per_head ? hm / G : hm;       /* KV head */
-  const int Gm = sh->per_head ? 1 : G;                 /* query heads of the mask */
-  const int64_t h0 = sh->per_head ? hm : hm * G;       /* first of them */
-  const int64_t i0 = qb * sh->block_q, i1 = min64(i0 + sh->block_q, sh->q_len);
-  const int64_t q_first = sh->q_pos0 + i0, q_last = sh->q_pos0 + i1 - 1;
-  const int64_t Tc = min64(q_last + 1, sh->seq_len);
-  const int64_t N = cdiv64(Tc, bk);
-  const int64_t n0 = min64(sh->topk / bk, N);
+  const int d = sh->head_dim;
+  const int64_t bk = sh->block_k;
+  unit_rows u;
+  if (unit_setup(sh, unit, &u) != OR_OK) return OR_BAD;
+  const int64_t q_first = u.q_first, q_last = u.q_last;
+  const int64_t N = u.N, n0 = u.n0;
   const int64_t cap = oracle_idx_cap(sh);
 
   cand* chunks = (cand*)malloc(sizeof(cand) * (size_t)n0);
@@ -214,21 +274,7 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
     scored += nc;
     for (int64_t c = 0; c < nc; ++c) {
       int64_t rep = cands[c].s + (cands[c].e - cands[c].s) / 2;
-      float best = -INFINITY;
-      for (int h = 0; h < Gm; ++h) {
-        const int64_t qh = h0 + h;
-        for (int64_t i = i0; i < i1; ++i) {
-          const int64_t p = sh->q_pos0 + i;
-          const float* qr = q + (((b * sh->n_qheads + qh) * sh->q_len + i) * d);
-          for (int64_t j = rep * bk; j < min64(rep * bk + bk, Tc); ++j) {
-            if (j > p) continue;
-            const float* kj = k + (((b * sh->n_kvheads + g) * sh->kv_capacity + j) * d);
-            float sc = oracle_canonical_dot(qr, kj, d);
-            if (sc > best) best = sc;
-          }
-        }
-      }
-      cands[c].score = best;
+      cands[c].score = block_score(q, k, sh, &u, rep);
     }
     /* step 4: global top-n0 of all candidates */
     qsort(cands, (size_t)nc, sizeof(cand), cand_order);

@@ -75,3 +75,17 @@ def test_oracle_inputs_decode_e5m2_and_pass_others_through():
     np.testing.assert_array_equal(out["k"], np.array([[1.0, -2.0]], np.float32))
     np.testing.assert_array_equal(out["v"], np.array([[2.0, 2.0 ** -16]], np.float32))
     assert bench.oracle_inputs(W.DECODE_128K, x) is x
+
+
+def test_layer_buffers_outgrow_the_l2_by_the_bytes_a_step_touches():
+    # decode at 128k touches ~63 MB per step (six rounds of 2048 two-key
+    # candidates per KV head, then ~1600 attended blocks of K and V): at
+    # least 4x the 126 MB L2 between two uses of a layer takes 9 layers
+    w = W.DECODE_128K
+    t = bench.touched_bytes(w)
+    assert t == 8 * (6 * 2048 + 2 * (1024 + 64 + 513)) * 2 * 128 * 2
+    n = bench.layer_count(w, 537 << 20, 0)
+    assert n * t >= 4 * bench.L2_BYTES and (n - 1) * t < 4 * bench.L2_BYTES
+    # prefill reads all of q, k and v; a requested count is kept
+    assert bench.touched_bytes(W.PREFILL_32K) == (2 * 8 + 32) * 32768 * 128 * 2
+    assert bench.layer_count(W.PREFILL_32K, 400 << 20, 5) == 5

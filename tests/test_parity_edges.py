@@ -2,8 +2,8 @@
 a prefill chunk whose query rows start after the first key (q_pos0 > 0),
 caches of one to a few keys, sink and window longer than the cache, a
 budget larger than the cache in prefill, and decode groups through the
-one-call entry point. Masks must match the oracle bit-exactly (up to the
-near-tie rule); attention is compared on the oracle's idx."""
+one-call entry point. Masks must match the oracle bit-exactly; attention is
+compared on the oracle's idx and end to end on the GPU's idx."""
 import numpy as np
 import pytest
 
@@ -43,13 +43,16 @@ def _run(x_q, x_k, x_v, dtype, *, batch, hq, hkv, T, q_len, q_pos0, bq, bk, topk
     idx_ref, gap, _ = oracle.mask(x_q, x_k, osh)
     idx_ref_dev = torch.from_numpy(idx_ref).cuda().reshape(idx.shape).contiguous()
     out = s.sparse_attn(q, k, v, idx_ref_dev)
+    if out_f is None:
+        out_f = s.sparse_attn(q, k, v, idx)  # end to end through the two calls
     torch.cuda.synchronize()
     s.check()
-    st = pu.compare_masks(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref, gap)
+    ig = idx.cpu().numpy().reshape(idx_ref.shape)
+    pu.compare_masks(ig, idx_ref, gap, validate=pu.gpu_validator(x_q, x_k, osh, s, q, k))
     ref = oracle.attention(x_q, x_k, x_v, idx_ref, osh)
     pu.compare_outputs(out.float().cpu().numpy().reshape(ref.shape), ref, dtype)
-    if out_f is not None and st["mismatched"] == 0:
-        pu.compare_outputs(out_f.float().cpu().numpy().reshape(ref.shape), ref, dtype)
+    ref_g = ref if np.array_equal(ig, idx_ref) else oracle.attention(x_q, x_k, x_v, ig, osh)
+    pu.compare_outputs(out_f.float().cpu().numpy().reshape(ref.shape), ref_g, dtype)
     return idx_ref
 
 
