@@ -78,7 +78,39 @@ struct MaskPlan {
   size_t ws;
   bool mma;  // tensor-core kernel (bf16 or e5m2 keys) or CUDA-core kernel
   bool norms;  // key-block norm pre-pass into the workspace (many-row masks)
+  bool decode;  // the decode kernel (one query position per mask row)
 };
+
+// Decode plan: e5m2 keys, one query position per mask row (b_q = 1, or a
+// single query row) with at most decode_max_rows() query rows. A cluster
+// of C CTAs per mask row (C the largest size with every row resident at once,
+// at least 8 candidates per CTA); the attention, when asked for, runs in the
+// same launch.
+int plan_decode(const hips_params* p, int cluster_cap, bool attend, MaskPlan* plan) {
+  hips::MaskArgs& a = plan->a;
+  if (p->dtype != HIPS_BF16_E5M2 || !(p->q_len == 1 || p->block_q == 1) ||
+      a.rows_max > hips::decode_max_rows() || a.units > 65535)
+    return HIPS_ERR_UNSUPPORTED;
+  const int64_t ncand = 2 * static_cast<int64_t>(a.n0max);
+  int c = 1;
+  for (int t = std::min(cluster_cap, 16); t > 1; --t) {
+    if (a.units * t <= kPlanSMs && cdiv(ncand, t) >= 8) {
+      c = t;
+      break;
+    }
+  }
+  a.cluster = c;
+  a.per_cta = static_cast<int>(cdiv(cdiv(ncand, c), 8) * 8);
+  a.rows_pad = a.rows_max;
+  a.stages = 0;
+  plan->smem = hips::decode_smem_bytes(a, attend, kMaxSmem);
+  if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
+  plan->decode = true;
+  plan->mma = false;
+  plan->norms = false;
+  plan->ws = kStatusBytes;
+  return HIPS_OK;
+}
 
 // Tensor-core mask plan: bf16 keys with up to 256 query rows per mask, or
 // e5m2 keys with up to 16 (one MMA column block); b_k <= 32.
@@ -120,9 +152,10 @@ int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   return HIPS_OK;
 }
 
-int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
+int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan, bool attend = false) {
   hips::MaskArgs& a = plan->a;
   a = hips::MaskArgs{};
+  plan->decode = false;
   a.dtype = p->dtype;
   a.n_qheads = p->n_qheads;
   a.n_kvheads = mask_heads(p);
@@ -144,8 +177,14 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   a.rows_max = group_rows(p, p->block_q);
   plan->mma = false;
   plan->norms = false;
+  // The tensor-core mask kernel first: it is the faster one wherever it
+  // plans (measured at 128k and 1M keys, one and 16 sequences). The decode
+  // kernel serves the e5m2 decode shapes it cannot plan (budgets whose
+  // candidate lists outgrow its shared memory).
   if (plan_mask_mma(p, cluster_cap, plan) == HIPS_OK) return HIPS_OK;
-  if (p->dtype == HIPS_BF16_E5M2) return HIPS_ERR_UNSUPPORTED;  // no CUDA-core e5m2 mask
+  if (plan_decode(p, cluster_cap, attend, plan) == HIPS_OK) return HIPS_OK;
+  plan->decode = false;
+  if (p->dtype == HIPS_BF16_E5M2) return HIPS_ERR_UNSUPPORTED;  // no other e5m2 mask
   if (a.rows_max > 32 || a.units > 65535) return HIPS_ERR_UNSUPPORTED;
   const int rc = hips::mask_fma_rc(a.rows_max);
   a.rows_pad = static_cast<int>(cdiv(a.rows_max, rc) * rc);
@@ -179,15 +218,18 @@ int resident_clusters(const MaskPlan& plan) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   const hips::MaskArgs& a = plan.a;
-  const int rows = plan.mma ? 100 + hips::mask_mma_nc(a.rows_max) : hips::mask_fma_rc(a.rows_max);
+  const int rows = plan.decode ? 200 + a.rows_max
+                   : plan.mma  ? 100 + hips::mask_mma_nc(a.rows_max)
+                               : hips::mask_fma_rc(a.rows_max);
   for (int i = 0; i < used; ++i) {
     const Entry& e = cache[i];
     if (e.dev == dev && e.dtype == a.dtype && e.rows == rows && e.cluster == a.cluster &&
         e.smem == plan.smem)
       return e.n;
   }
-  const int n = plan.mma ? hips::mask_mma_max_active_clusters(a, plan.smem)
-                         : hips::mask_fma_max_active_clusters(a, plan.smem);
+  const int n = plan.decode ? hips::decode_max_active_clusters(a, plan.smem)
+                : plan.mma  ? hips::mask_mma_max_active_clusters(a, plan.smem)
+                            : hips::mask_fma_max_active_clusters(a, plan.smem);
   if (used < 64) cache[used++] = Entry{dev, a.dtype, rows, a.cluster, plan.smem, n};
   return n;
 }
@@ -320,8 +362,8 @@ int run_attention(const void* q, const void* k, const void* v, const int32_t* id
 // launch for a decode step) when the row group is a single MMA column block
 // of at most mask_mma_fused_rows() query rows.
 bool fusable(const MaskPlan& plan) {
-  return plan.mma && hips::mask_mma_nc(plan.a.rows_max) == 1 &&
-         plan.a.rows_max <= hips::mask_mma_fused_rows();
+  return plan.decode || (plan.mma && hips::mask_mma_nc(plan.a.rows_max) == 1 &&
+                         plan.a.rows_max <= hips::mask_mma_fused_rows());
 }
 
 // Plan and launch the mask kernel (with the fused attention when v and out
@@ -331,13 +373,14 @@ bool fusable(const MaskPlan& plan) {
 int launch_mask(const void* q, const void* k, const hips_params* params, int32_t* idx_out,
                 const void* v, void* out) {
   MaskPlan plan;
-  int st = plan_mask(params, 16, &plan);
+  const bool attend = out != nullptr;
+  int st = plan_mask(params, 16, &plan, attend);
   if (st) return st;
   st = check_workspace(params, plan.ws);
   if (st) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
   for (int cap = 16; cap >= 1; cap = std::min(cap - 1, plan.a.cluster - 1)) {
-    st = plan_mask(params, cap, &plan);
+    st = plan_mask(params, cap, &plan, attend);
     if (st) return st;
     if (plan.a.cluster > cap) continue;
     if (plan.a.cluster > 1 && cap > 1) {
@@ -358,8 +401,9 @@ int launch_mask(const void* q, const void* k, const hips_params* params, int32_t
       a.out = out;
       a.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
     }
-    const cudaError_t e = plan.mma ? hips::launch_mask_mma(a, plan.smem, stream)
-                                   : hips::launch_mask_fma(a, plan.smem, stream);
+    const cudaError_t e = plan.decode ? hips::launch_decode(a, plan.smem, stream)
+                          : plan.mma  ? hips::launch_mask_mma(a, plan.smem, stream)
+                                      : hips::launch_mask_fma(a, plan.smem, stream);
     if (e == cudaSuccess) return HIPS_OK;
     if ((e == cudaErrorInvalidClusterSize || e == cudaErrorLaunchOutOfResources) && cap > 1) {
       (void)cudaGetLastError();
@@ -463,7 +507,7 @@ int hip_mask_sparse_attn(const void* q, const void* k, const void* v, const hips
     return HIPS_ERR_INVALID_ARG;
   if (params->mask_len != params->seq_len) return HIPS_ERR_INVALID_ARG;  // a fresh mask
   MaskPlan plan;
-  st = plan_mask(params, 16, &plan);
+  st = plan_mask(params, 16, &plan, true);
   if (st) return st;
   if (fusable(plan)) return launch_mask(q, k, params, idx_out, v, out);
   st = launch_mask(q, k, params, idx_out, nullptr, nullptr);

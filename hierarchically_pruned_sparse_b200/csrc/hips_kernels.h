@@ -42,6 +42,11 @@ struct MaskArgs {
   // block's key 2-norms, written by key_block_norms before the mask launch
   const float* knorm;
   int64_t knorm_stride;  // key blocks per head (ceil(seq_len / block_k))
+  // decode kernel: keep the last round's dots for the attention; bytes of
+  // one slot of its staging ring
+  int stash_dots;
+  int slot_bytes;
+  int list_cap;  // entries of its staging list
 };
 
 struct AttnArgs {
@@ -78,6 +83,15 @@ cudaError_t launch_mask_mma(const MaskArgs& a, int smem, cudaStream_t stream);
 int mask_mma_fused_rows();  // most query rows of a fused mask + attention launch
 // Fill a.knorm (a workspace array of units' heads x knorm_stride floats)
 cudaError_t launch_key_block_norms(const MaskArgs& a, int batch, cudaStream_t stream);
+
+// Decode-shaped masks over e5m2 keys (one query position per mask row, at
+// most decode_max_rows() query rows) with their attention, on CUDA cores
+// (decode.cu). decode_smem_bytes sets a.stash_dots (the last round's dots
+// kept for the attention) and a.slot_bytes (staging ring) within smem_cap.
+int decode_max_rows();
+int decode_smem_bytes(MaskArgs& a, bool attend, int smem_cap);
+int decode_max_active_clusters(const MaskArgs& a, int smem);
+cudaError_t launch_decode(const MaskArgs& a, int smem, cudaStream_t stream);
 
 // Tensor-core attention for query blocks, bf16 (attn_mma.cu)
 int attn_mma_smem_bytes(int table_items);

@@ -86,11 +86,11 @@ enum hips_status {
  * command of the SGLang pull request "[Feature] Support Efficient Sparse HiP
  * Attention (InfiniteHiP)"), while q and out are bf16. Every code widens
  * exactly to bf16, and the mask and attention are those of bf16 keys and
- * values with the widened values. Supported for masks of at most 16 query
- * rows (decode: G heads x b_q <= 16) with block_k <= 32 and topk / block_k
- * <= 1024, and for attention of at most 8 rows per query block; other
- * shapes return HIPS_ERR_UNSUPPORTED (from the call and as a zero
- * hip_workspace_size). */
+ * values with the widened values. Supported for masks of one query position
+ * per mask row (decode, or b_q = 1) with at most 8 query rows, for masks of
+ * 9 to 16 query rows with block_k <= 32 and topk / block_k <= 1024, and for
+ * attention of at most 8 rows per query block; other shapes return
+ * HIPS_ERR_UNSUPPORTED (from the call and as a zero hip_workspace_size). */
 enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1, HIPS_BF16_E5M2 = 2 };
 
 enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2, HIPS_OP_MASK_SPARSE = 3 };

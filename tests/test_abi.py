@@ -153,10 +153,12 @@ def test_e5m2_kv_plans_decode_and_rejects_other_shapes():
                     window=1024)
     assert hb.workspace_size(pre, hb.OP_MASK) == 0
     assert hb.workspace_size(pre, hb.OP_SPARSE) == 0
-    # more than 1024 chunks per mask does not fit beside the staging tiles
+    # 2048 chunks per mask do not fit beside the tensor-core kernel's tiles:
+    # e5m2 decode masks (one query position, at most 8 rows) then run on the
+    # CUDA-core decode kernel, bf16 ones on the CUDA-core mask kernel
     big = _decode_params(dtype=hb.HIPS_BF16_E5M2, topk=4096)
-    assert hb.workspace_size(big, hb.OP_MASK) == 0
-    assert hb.workspace_size(_decode_params(topk=4096), hb.OP_MASK) >= 256  # bf16 has a kernel
+    assert hb.workspace_size(big, hb.OP_MASK) >= 256
+    assert hb.workspace_size(_decode_params(topk=4096), hb.OP_MASK) >= 256
 
 
 @pytest.mark.parametrize("name", sorted(W.WORKLOADS))

@@ -82,6 +82,11 @@ SMALL = [
     (W.Workload("e2", "decode", 2, 16, 2, 128, 3001, 1, 4, 128, 0, 32, "e5m2", 2, "uniform"), True),
     # a cache of a few keys (fewer than one budget)
     (W.Workload("e4", "decode", 1, 4, 2, 128, 7, 1, 2, 4, 0, 0, "e5m2"), True),
+    # 2048 chunks per mask: more than the tensor-core mask kernel holds, so
+    # the CUDA-core decode kernel plans it (one launch, 4 rows, ragged T)
+    (W.Workload("e5", "decode", 1, 4, 1, 128, 20011, 1, 2, 4096, 16, 256, "e5m2", 4, "uniform"), True),
+    # the same kernel for the mask alone: 8 rows, b_k = 4, batch of 2
+    (W.Workload("e6", "decode", 2, 16, 2, 128, 9001, 1, 4, 8192, 0, 64, "e5m2", 2, "uniform"), False),
 ]
 
 
