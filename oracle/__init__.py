@@ -33,6 +33,13 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+class Stage(ctypes.Structure):
+    """Mirror of ``oracle_stage`` in hip_oracle.c: one pruning stage."""
+
+    _fields_ = [("chunk_size", ctypes.c_int32), ("stage_k", ctypes.c_int32),
+                ("stride_q", ctypes.c_int32), ("pad", ctypes.c_int32)]
+
+
 class Shape(ctypes.Structure):
     """Mirror of ``oracle_shape`` in hip_oracle.c."""
 
@@ -45,6 +52,7 @@ class Shape(ctypes.Structure):
         ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("topk", ctypes.c_int32), ("sink", ctypes.c_int32),
         ("window", ctypes.c_int32), ("per_head", ctypes.c_int32),
+        ("n_stages", ctypes.c_int32), ("stages", ctypes.POINTER(Stage)),
     ]
 
 
@@ -94,14 +102,21 @@ def _f32(a) -> np.ndarray:
 
 
 def shape(*, batch, n_qheads, n_kvheads, head_dim, seq_len, q_len, q_pos0, block_q,
-          block_k, topk, sink=0, window=0, mask_len=None, kv_capacity=None, per_head=0) -> Shape:
+          block_k, topk, sink=0, window=0, mask_len=None, kv_capacity=None, per_head=0,
+          stages=()) -> Shape:
     """per_head=1: one mask per query head (idx rows [B, Hq, n_qblocks]) instead of
-    one per KV-head group."""
-    return Shape(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, head_dim=head_dim,
-                 seq_len=seq_len, mask_len=seq_len if mask_len is None else mask_len,
-                 kv_capacity=seq_len if kv_capacity is None else kv_capacity,
-                 q_len=q_len, pad0=0, q_pos0=q_pos0, block_q=block_q, block_k=block_k,
-                 topk=topk, sink=sink, window=window, per_head=int(per_head))
+    one per KV-head group. stages: (chunk_size, stage_k, stride_q) per pruning
+    stage before the iteration (stage_k 0 keeps every chunk); topk is then
+    the iteration's budget (second_stage_k)."""
+    st = (Stage * max(1, len(stages)))(*[Stage(int(c), int(k), int(r), 0) for c, k, r in stages])
+    sh = Shape(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, head_dim=head_dim,
+               seq_len=seq_len, mask_len=seq_len if mask_len is None else mask_len,
+               kv_capacity=seq_len if kv_capacity is None else kv_capacity,
+               q_len=q_len, pad0=0, q_pos0=q_pos0, block_q=block_q, block_k=block_k,
+               topk=topk, sink=sink, window=window, per_head=int(per_head),
+               n_stages=len(stages), stages=ctypes.cast(st, ctypes.POINTER(Stage)))
+    sh._stage_array = st  # keeps the stage list alive with the shape
+    return sh
 
 
 def set_threads(n: int = 0) -> int:

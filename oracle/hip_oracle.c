@@ -27,6 +27,15 @@
  *            Specification", E5M2): 1 sign bit, 5 exponent bits with bias 15,
  *            2 mantissa bits; exponent 0 holds zero and the subnormals
  *            m/4 * 2^-14, exponent 31 the infinities (m = 0) and NaNs.
+ *            The same commands configure InfiniteHiP's multi-stage pruning
+ *            (--hip-attention-config): per layer a list of stages, each with
+ *            stage_chunk_size, stage_k, stage_block_size_q,
+ *            stage_block_stride_q and stage_stride, then second_stage_k and
+ *            sliding_window_size.
+ *  [T2wK]    "A Training-free ... Hierarchically Pruned Attention", Author
+ *            Rebuttal to the Reviewer T2wK, Q1 (the latest HiP): the user
+ *            sets, per iteration, how many chunks are selected, how each
+ *            chunk is broken down and how its representative is chosen.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - chunk i of n0 over N blocks is [floor(iN/n0), floor((i+1)N/n0));
@@ -51,6 +60,22 @@
  *    the 8 lane partials are added as ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7));
  *  - sink = key blocks [0, ceil(sink/b_k)); window = the blocks covering keys
  *    [max(0, q_first-window+1), q_last] of the query block;
+ *  - stages ([PR], [T2wK]): stage 1 tiles the keys [0, T_c) into chunks of
+ *    stage_chunk_size keys aligned at multiples of it (a multiple of b_k,
+ *    the last chunk clipped); stage s > 1 cuts every chunk that survived
+ *    stage s-1 into pieces of its own chunk size (which divides the
+ *    previous one). A stage scores its chunks like the halves of the
+ *    iteration (centre block, max of the canonical dot) and keeps the
+ *    stage_k / stage_chunk_size best by (score desc, start asc); a stage_k
+ *    of 0 (null on the page) keeps every chunk unscored. The stage's query
+ *    rows are the mask's (stage_block_size_q read as the mask's b_q) taken
+ *    at stride stage_block_stride_q counted back from the block's last row,
+ *    which sees every key of the range. stage_stride is 1 throughout the
+ *    page's configuration and is not modelled. After the stages the
+ *    iteration above runs with k = second_stage_k from the surviving chunks
+ *    instead of the n0 uniform ones: halve, keep the top n0 (every candidate
+ *    when there are no more than n0), stop at single blocks. Without stages
+ *    it is the plain iteration;
  *  - attention of a query at position p uses the keys j of the selected
  *    blocks with j <= p and j < mask_len, plus every key in
  *    [mask_len, seq_len) with j <= p (keys appended since the mask refresh).
@@ -74,7 +99,17 @@ typedef struct {
   int64_t q_pos0;       /* absolute position of query row 0 */
   int32_t block_q, block_k, topk, sink, window;
   int32_t per_head;     /* 1: one mask per query head, not per KV-head group */
+  int32_t n_stages;     /* pruning stages before the iteration (0: none) */
+  const struct oracle_stage* stages;
 } oracle_shape;
+
+/* One pruning stage ([PR], [T2wK]; readings in the header). */
+typedef struct oracle_stage {
+  int32_t chunk_size;  /* keys per chunk: a multiple of b_k dividing the previous stage's */
+  int32_t stage_k;     /* keys kept (a multiple of chunk_size); 0 keeps every chunk */
+  int32_t stride_q;    /* query-row stride within the query block, >= 1 */
+  int32_t pad;
+} oracle_stage;
 
 enum { OR_OK = 0, OR_BAD = -1, OR_NOMEM = -2 };
 
@@ -137,6 +172,13 @@ static int shape_ok(const oracle_shape* s) {
   if (s->block_q <= 0 || s->block_k <= 0 || s->topk < s->block_k) return 0;
   if (s->topk % s->block_k || s->sink < 0 || s->window < 0) return 0;
   if (s->per_head != 0 && s->per_head != 1) return 0;
+  if (s->n_stages < 0 || (s->n_stages > 0 && !s->stages)) return 0;
+  for (int i = 0; i < s->n_stages; ++i) {
+    const oracle_stage* g = &s->stages[i];
+    if (g->chunk_size <= 0 || g->chunk_size % s->block_k || g->stride_q < 1) return 0;
+    if (g->stage_k < 0 || g->stage_k % g->chunk_size) return 0;
+    if (i > 0 && s->stages[i - 1].chunk_size % g->chunk_size) return 0;
+  }
   return 1;
 }
 
@@ -159,6 +201,18 @@ static int cand_order(const void* pa, const void* pb) {
   if (a->score > b->score) return -1;
   if (a->score < b->score) return 1;
   return (a->s > b->s) - (a->s < b->s);
+}
+
+/* [RsGC] step 4 (and a stage's selection): rank the nc scored candidates by
+ * (score desc, start asc) and keep the best m < nc as the new chunks;
+ * *gap takes the smaller of itself and the score gap at the cut, in
+ * q.k/sqrt(d) units. Returns m. */
+static int64_t rank_and_keep(cand* cands, int64_t nc, int64_t m, cand* chunks, int d, double* gap) {
+  qsort(cands, (size_t)nc, sizeof(cand), cand_order);
+  const double gp = ((double)cands[m - 1].score - (double)cands[m].score) / sqrt((double)d);
+  if (gp < *gap) *gap = gp;
+  for (int64_t i = 0; i < m; ++i) chunks[i] = cands[i];
+  return m;
 }
 
 /* The query rows and the key range of one mask row (unit). */
@@ -191,15 +245,16 @@ static int unit_setup(const oracle_shape* sh, int64_t unit, unit_rows* u) {
 
 /* [RsGC] step 3: the score of key block `rep` for the unit's query rows: the
  * max over the rows and the block's keys j < Tc, j <= p (causal) of the
- * canonical dot q.k; -inf when no row sees a key of the block. */
+ * canonical dot q.k; -inf when no row sees a key of the block. A stage
+ * scores with the rows i1-1, i1-1-stride, ... of the block (stride 1: all). */
 static float block_score(const float* q, const float* k, const oracle_shape* sh,
-                         const unit_rows* u, int64_t rep) {
+                         const unit_rows* u, int64_t rep, int stride) {
   const int d = sh->head_dim;
   const int64_t bk = sh->block_k;
   float best = -INFINITY;
   for (int h = 0; h < u->Gm; ++h) {
     const int64_t qh = u->h0 + h;
-    for (int64_t i = u->i0; i < u->i1; ++i) {
+    for (int64_t i = u->i1 - 1; i >= u->i0; i -= stride) {
       const int64_t p = sh->q_pos0 + i;
       const float* qr = q + (((u->b * sh->n_qheads + qh) * sh->q_len + i) * d);
       for (int64_t j = rep * bk; j < min64(rep * bk + bk, u->Tc); ++j) {
@@ -224,7 +279,7 @@ int oracle_block_scores(const float* q, const float* k, const oracle_shape* sh, 
   unit_rows u;
   if (unit_setup(sh, unit, &u) != OR_OK) return OR_BAD;
   for (int64_t i = 0; i < n; ++i)
-    out[i] = (blocks[i] >= 0 && blocks[i] < u.N) ? block_score(q, k, sh, &u, blocks[i]) : -INFINITY;
+    out[i] = (blocks[i] >= 0 && blocks[i] < u.N) ? block_score(q, k, sh, &u, blocks[i], 1) : -INFINITY;
   return OR_OK;
 }
 
@@ -242,25 +297,62 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
   const int64_t N = u.N, n0 = u.n0;
   const int64_t cap = oracle_idx_cap(sh);
 
-  cand* chunks = (cand*)malloc(sizeof(cand) * (size_t)n0);
-  cand* cands = (cand*)malloc(sizeof(cand) * (size_t)(2 * n0));
+  /* chunks and candidates never overlap, so N bounds both lists */
+  cand* chunks = (cand*)malloc(sizeof(cand) * (size_t)N);
+  cand* cands = (cand*)malloc(sizeof(cand) * (size_t)N);
   unsigned char* keep = (unsigned char*)calloc((size_t)N, 1);
   if (!chunks || !cands || !keep) { free(chunks); free(cands); free(keep); return OR_NOMEM; }
 
-  /* step 1: n0 chunks that tile the block range [0, N) */
-  for (int64_t i = 0; i < n0; ++i) {
-    chunks[i].s = i * N / n0;
-    chunks[i].e = (i + 1) * N / n0;
-  }
   double gap = INFINITY;
   int32_t rounds = 0;
-  int64_t scored = 0;
+  int64_t scored = 0, nk = 0; /* nk: chunks kept so far */
+
+  if (sh->n_stages == 0) {
+    /* step 1: n0 chunks that tile the block range [0, N) */
+    for (int64_t i = 0; i < n0; ++i) {
+      chunks[i].s = i * N / n0;
+      chunks[i].e = (i + 1) * N / n0;
+    }
+    nk = n0;
+  } else {
+    /* stage 1 cuts the whole range [0, N) into pieces of its chunk size, a
+     * later stage every survivor of the one before; a stage with stage_k > 0
+     * keeps its best stage_k / chunk_size pieces */
+    chunks[0].s = 0;
+    chunks[0].e = N;
+    nk = 1;
+    for (int st = 0; st < sh->n_stages; ++st) {
+      const oracle_stage* g = &sh->stages[st];
+      const int64_t cs = g->chunk_size / bk;
+      int64_t nc = 0;
+      for (int64_t i = 0; i < nk; ++i)
+        for (int64_t s0 = chunks[i].s; s0 < chunks[i].e; s0 += cs) {
+          cands[nc].s = s0;
+          cands[nc].e = min64(s0 + cs, chunks[i].e);
+          ++nc;
+        }
+      const int64_t m = g->stage_k / g->chunk_size;
+      if (g->stage_k > 0 && nc > m) {
+        for (int64_t c = 0; c < nc; ++c)
+          cands[c].score = block_score(q, k, sh, &u, cands[c].s + (cands[c].e - cands[c].s) / 2,
+                                       g->stride_q);
+        nk = rank_and_keep(cands, nc, m, chunks, d, &gap);
+        scored += nc;
+        ++rounds;
+      } else {
+        for (int64_t i = 0; i < nc; ++i) chunks[i] = cands[i];
+        nk = nc;
+      }
+    }
+  }
   for (;;) {
     int64_t nc = 0, longest = 0;
-    for (int64_t i = 0; i < n0; ++i) longest = max64(longest, chunks[i].e - chunks[i].s);
-    if (longest <= 1) break; /* every chunk is one b_k block: stop */
+    for (int64_t i = 0; i < nk; ++i) longest = max64(longest, chunks[i].e - chunks[i].s);
+    /* every chunk is one b_k block, no more of them than n0: stop (stages
+     * may leave more single blocks than n0; they are ranked once more) */
+    if (longest <= 1 && nk <= n0) break;
     /* step 2: halve every chunk */
-    for (int64_t i = 0; i < n0; ++i) {
+    for (int64_t i = 0; i < nk; ++i) {
       int64_t s = chunks[i].s, e = chunks[i].e, L = e - s;
       if (L > 1) {
         int64_t m = s + L / 2;
@@ -270,22 +362,23 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
         cands[nc].s = s; cands[nc].e = e; ++nc;
       }
     }
+    if (nc <= n0) {
+      /* no more candidates than survivors: all are kept, none is ranked */
+      for (int64_t i = 0; i < nc; ++i) chunks[i] = cands[i];
+      nk = nc;
+      continue;
+    }
     /* step 3: score each half by its centre block */
-    scored += nc;
     for (int64_t c = 0; c < nc; ++c) {
       int64_t rep = cands[c].s + (cands[c].e - cands[c].s) / 2;
-      cands[c].score = block_score(q, k, sh, &u, rep);
+      cands[c].score = block_score(q, k, sh, &u, rep, 1);
     }
     /* step 4: global top-n0 of all candidates */
-    qsort(cands, (size_t)nc, sizeof(cand), cand_order);
-    if (nc > n0) {
-      double gp = ((double)cands[n0 - 1].score - (double)cands[n0].score) / sqrt((double)d);
-      if (gp < gap) gap = gp;
-    }
-    for (int64_t i = 0; i < n0; ++i) chunks[i] = cands[i];
+    nk = rank_and_keep(cands, nc, n0, chunks, d, &gap);
+    scored += nc;
     ++rounds;
   }
-  for (int64_t i = 0; i < n0; ++i) keep[chunks[i].s] = 1;
+  for (int64_t i = 0; i < nk; ++i) keep[chunks[i].s] = 1;
   /* always-kept sink and sliding-window blocks */
   for (int64_t c = 0; c < min64(cdiv64(sh->sink, bk), N); ++c) keep[c] = 1;
   if (sh->window > 0) {
@@ -293,6 +386,9 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
     for (int64_t c = lo / bk; c <= q_last / bk && c < N; ++c) keep[c] = 1;
   }
   int64_t nnz = 0;
+  for (int64_t c = 0; c < N; ++c) nnz += keep[c];
+  if (nnz > cap) { free(chunks); free(cands); free(keep); return OR_BAD; }
+  nnz = 0;
   for (int64_t c = 0; c < N; ++c)
     if (keep[c]) row[1 + nnz++] = (int32_t)c;
   row[0] = (int32_t)nnz;
@@ -301,7 +397,7 @@ static int mask_unit(const float* q, const float* k, const oracle_shape* sh, int
   if (rounds_out) *rounds_out = rounds;
   if (scored_out) *scored_out = scored;
   free(chunks); free(cands); free(keep);
-  return nnz <= cap ? OR_OK : OR_BAD;
+  return OR_OK;
 }
 
 /*

@@ -32,8 +32,8 @@ MUTANTS = [
     ("tree_order", "float a0 = part[0] + part[4], a1 = part[1] + part[5];",
      "float a0 = part[0] + part[1], a1 = part[4] + part[5];"),
     ("causal_bound", "if (j > p) continue;", "if (j > p + 1) continue;"),
-    ("chunk_tiling", "chunks[i].s = i * N / n0;\n    chunks[i].e = (i + 1) * N / n0;",
-     "chunks[i].s = (i * N + n0 - 1) / n0;\n    chunks[i].e = ((i + 1) * N + n0 - 1) / n0;"),
+    ("chunk_tiling", "chunks[i].s = i * N / n0;\n      chunks[i].e = (i + 1) * N / n0;",
+     "chunks[i].s = (i * N + n0 - 1) / n0;\n      chunks[i].e = ((i + 1) * N + n0 - 1) / n0;"),
     ("reuse_tail",
      "for (int64_t j = sh->mask_len; j < sh->seq_len && j <= p; ++j) keys[n++] = j;",
      "for (int64_t j = sh->mask_len; j + 1 < sh->seq_len && j <= p; ++j) keys[n++] = j;"),
@@ -47,7 +47,18 @@ MUTANTS = [
      "const double scale = 1.0 / sqrt((double)d + 1);"),
     ("attn_drop_first_weight", "    l += w;\n", "    l += (t ? w : 0.0);\n"),
     ("gqa_head", "u->h0 = sh->per_head ? hm : hm * G;", "u->h0 = sh->per_head ? hm : hm;"),
-    ("stop_early", "if (longest <= 1) break;", "if (longest <= 2) break;"),
+    ("stop_early", "if (longest <= 1 && nk <= n0) break;", "if (longest <= 2 && nk <= n0) break;"),
+    ("stage_keep_count", "const int64_t m = g->stage_k / g->chunk_size;",
+     "const int64_t m = g->stage_k / g->chunk_size + 1;"),
+    ("stage_rows_from_first", "for (int64_t i = u->i1 - 1; i >= u->i0; i -= stride) {",
+     "for (int64_t i = u->i0; i < u->i1; i += stride) {"),
+    ("stage_chunk_in_keys", "const int64_t cs = g->chunk_size / bk;",
+     "const int64_t cs = g->chunk_size;"),
+    ("stage_stride_dropped", "                                       g->stride_q);",
+     "                                       1);"),
+    ("stage_rep_start", "cands[c].score = block_score(q, k, sh, &u, cands[c].s + (cands[c].e - cands[c].s) / 2,",
+     "cands[c].score = block_score(q, k, sh, &u, cands[c].s + (cands[c].e - cands[c].s - 1) / 2,"),
+    ("single_blocks_over_budget", "if (longest <= 1 && nk <= n0) break;", "if (longest <= 1) break;"),
     ("per_head_kv_map", "u->g = sh->per_head ? hm / G : hm;",
      "u->g = sh->per_head ? hm % sh->n_kvheads : hm;"),
     ("per_head_idx_row", "const int64_t mrow = sh->per_head ? b * sh->n_qheads + h : b * sh->n_kvheads + g;",

@@ -8,7 +8,10 @@
 * closed forms (monotone keys keep the last blocks; equal keys keep the
   first blocks through the tie rule) and the count invariant;
 * the canonical fp32 dot: exact on one-hot inputs, within the fp32
-  rounding bound of the exact dot, and the hand-derived order example.
+  rounding bound of the exact dot, and the hand-derived order example;
+* multi-stage pruning (InfiniteHiP stages): brute force on random schedules,
+  a single keep-all stage of the initial chunks equals the plain iteration,
+  and the monotone / equal-key closed forms through a three-stage schedule.
 """
 import math
 import os
@@ -474,3 +477,145 @@ def test_e5m2_generator_codes_round_to_nearest():
     got = oracle.decode_e5m2(codes).astype(np.float64)
     best = np.min(np.abs(table[finite][None, :] - x[:, None].astype(np.float64)), axis=1)
     assert np.all(np.abs(got - x) <= best * (1 + 1e-12))
+
+
+# ---------------------------------------------------------------- stages
+# The stage schedule of "[Feature] Support Efficient Sparse HiP Attention
+# (InfiniteHiP)" (serving command, --hip-attention-config): per stage a chunk
+# size, a stage_k (null: keep all) and a query-row stride; second_stage_k is
+# the iteration's budget (topk here).
+
+
+def _schedule(rng, bk, T, bq):
+    """1-3 stages; chunk sizes multiples of b_k, each dividing the previous;
+    stage_k 0 (keep all) or a multiple of the chunk size; random strides."""
+    sizes = [bk * int(rng.choice([1, 2, 3, 4]))]
+    for _ in range(int(rng.integers(0, 3))):
+        sizes.insert(0, sizes[0] * int(rng.choice([1, 2, 4])))
+    out = []
+    for c in sizes:
+        keep = 0 if rng.random() < 0.3 else c * int(rng.integers(1, max(2, T // c + 2)))
+        out.append((c, keep, int(rng.choice([1, 2, 3, bq]))))
+    return tuple(out)
+
+
+def _stage_cases():
+    rng = np.random.default_rng(23)
+    cases = []
+    for T in (5, 16, 33, 100, 257, 600):
+        for bk in (1, 2, 4):
+            for _ in range(2):
+                kind = "decode" if rng.random() < 0.5 else "prefill"
+                Lq = 1 if kind == "decode" else min(T, 48)
+                bq = 1 if kind == "decode" else int(rng.choice([4, 8, 16]))
+                G = int(rng.choice([1, 2]))
+                nb = -(-T // bk)
+                topk = bk * int(rng.integers(1, max(2, nb // 2 + 2)))
+                sink = int(rng.choice([0, 0, bk, 5]))
+                window = int(rng.choice([0, 0, 3, 2 * bk + 1]))
+                cases.append((T, bk, topk, kind, Lq, bq, G, sink, window, _schedule(rng, bk, T, bq)))
+    return cases
+
+
+@pytest.mark.parametrize("case", _stage_cases())
+def test_staged_mask_matches_brute_force_on_exact_scores(case):
+    T, bk, topk, kind, Lq, bq, G, sink, window, stages = case
+    rng = np.random.default_rng(zlib.crc32(repr(case).encode()))
+    B, Hkv = 1, 2
+    q, k = _int_inputs(rng, B, Hkv * G, Hkv, Lq, T)
+    q_pos0 = T - Lq
+    sh = _shape(batch=B, n_qheads=Hkv * G, n_kvheads=Hkv, head_dim=64, seq_len=T, q_len=Lq,
+                q_pos0=q_pos0, block_q=bq, block_k=bk, topk=topk, sink=sink, window=window,
+                stages=stages)
+    idx, gap, rounds = oracle.mask(q, k, sh)
+    nqb = -(-Lq // bq)
+    units = [(b, g, qb) for b in range(B) for g in range(Hkv) for qb in range(nqb)]
+    for u, (b, g, qb) in enumerate(units):
+        want, want_gap, want_rounds = bf.mask_row(
+            q, k, b=b, g=g, qb=qb, group=G, block_q=bq, block_k=bk, topk=topk, q_len=Lq,
+            q_pos0=q_pos0, seq_len=T, sink=sink, window=window, stages=stages)
+        row = idx[u]
+        assert list(row[1:1 + row[0]]) == want, (case, u)
+        assert rounds[u] == want_rounds, (case, u)
+        if math.isinf(want_gap):
+            assert math.isinf(gap[u])
+        else:
+            assert gap[u] == pytest.approx(want_gap / math.sqrt(64), rel=1e-12, abs=0)
+
+
+@pytest.mark.parametrize("T,bk,topk", [(4096, 2, 256), (8192, 4, 512), (2048, 1, 64)])
+def test_one_keep_all_stage_of_the_initial_chunks_is_the_plain_iteration(T, bk, topk):
+    # n0 divides N: the plain iteration's n0 initial chunks are the aligned
+    # chunks of b_k N / n0 keys, so a stage of that size that keeps every
+    # chunk (stage_k null, or at least T) leaves the iteration unchanged
+    rng = np.random.default_rng(T + bk)
+    d, G = 128, 4
+    q = rng.standard_normal((1, G, 1, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    N, n0 = T // bk, topk // bk
+    assert N % n0 == 0
+    base = dict(batch=1, n_qheads=G, n_kvheads=1, head_dim=d, seq_len=T, q_len=1,
+                q_pos0=T - 1, block_q=1, block_k=bk, topk=topk, sink=bk, window=3 * bk)
+    want = oracle.mask(q, k, _shape(**base), with_scored=True)
+    for keep in (0, T):
+        got = oracle.mask(q, k, _shape(**base, stages=((bk * N // n0, keep, 1),)), with_scored=True)
+        for a, b in zip(got, want):
+            np.testing.assert_array_equal(a, b)
+
+
+# a schedule shaped like the serving command's (chunks of 128, 32 and 8
+# keys; the first keeps all, the others a quarter of the range each time)
+PR_LIKE = ((128, 0, 4), (32, 2048, 4), (8, 512, 1))
+
+
+@pytest.mark.parametrize("T", [8192, 8000])
+def test_staged_monotone_keys_keep_last_blocks(T):
+    # every stage and round keeps its right-most chunks: the last n0 blocks
+    d, bk, topk = 128, 2, 256
+    q = np.ones((1, 2, 1, d), np.float32)
+    k = np.ascontiguousarray(np.broadcast_to(((np.arange(T) + 1) / T).astype(np.float32)[:, None],
+                                             (T, d)))[None, None]
+    sh = _shape(batch=1, n_qheads=2, n_kvheads=1, head_dim=d, seq_len=T, q_len=1,
+                q_pos0=T - 1, block_q=1, block_k=bk, topk=topk, stages=PR_LIKE)
+    idx, _, rounds, scored = oracle.mask(q, k, sh, with_scored=True)
+    N, n0 = -(-T // bk), topk // bk
+    assert list(idx[0, 1:1 + idx[0, 0]]) == list(range(N - n0, N))
+    # ranked: stages 2 and 3, then the rounds from 64 chunks of 4 blocks:
+    # halves (128 = n0, kept unranked), then 256 single blocks
+    assert rounds[0] == 3
+    assert scored[0] == -(-T // 32) + 512 // 8 * 4 + 256
+
+
+def test_staged_equal_keys_keep_first_blocks():
+    # every score ties: the lower start wins each time, down to [0, n0)
+    d, T, bk, topk = 128, 8192, 2, 256
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, 1, 1, d)).astype(np.float32)
+    k = np.ascontiguousarray(np.broadcast_to(rng.standard_normal(d).astype(np.float32), (T, d)))
+    sh = _shape(batch=1, n_qheads=1, n_kvheads=1, head_dim=d, seq_len=T, q_len=1,
+                q_pos0=T - 1, block_q=1, block_k=bk, topk=topk, stages=PR_LIKE)
+    idx, gap, _ = oracle.mask(q, k[None, None], sh)
+    assert list(idx[0, 1:1 + idx[0, 0]]) == list(range(topk // bk))
+    assert gap[0] == 0.0
+
+
+def test_stage_rows_are_counted_back_from_the_last_row():
+    # one query block of 4 rows at stride 4: only the last row scores the
+    # stage, so a key block that only the first row favours is pruned
+    d, T, bk = 64, 64, 4
+    q = np.zeros((1, 1, 4, d), np.float32)
+    k = np.zeros((1, 1, T, d), np.float32)
+    q[0, 0, 0, 0] = 1.0    # row 0 (position 60) wants dimension 0
+    q[0, 0, 3, 1] = 1.0    # row 3 (position 63) wants dimension 1
+    k[0, 0, 8, 0] = 5.0    # block 2 (chunk [0, 4) of 4 blocks) matches row 0
+    k[0, 0, 40, 1] = 1.0   # block 10 (chunk [8, 12)) matches row 3
+    base = dict(batch=1, n_qheads=1, n_kvheads=1, head_dim=d, seq_len=T, q_len=4, q_pos0=T - 4,
+                block_q=4, block_k=bk, topk=bk * 4)
+    rep = lambda c: c * 4 + 2  # noqa: E731 -- the centre block of chunk c
+    k[0, 0, rep(0) * bk, 0] = 5.0
+    k[0, 0, rep(2) * bk, 1] = 1.0
+    for stride, want_chunk in ((4, 2), (1, 0)):
+        sh = _shape(**base, stages=((16, 16, stride),))
+        idx, _, _ = oracle.mask(q, k, sh)
+        kept = list(idx[0, 1:1 + idx[0, 0]])
+        assert kept == list(range(want_chunk * 4, want_chunk * 4 + 4)), (stride, kept)
