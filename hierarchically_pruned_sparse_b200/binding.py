@@ -17,6 +17,8 @@ HIPS_ERR_WORKSPACE = -3
 HIPS_ERR_CUDA = -4
 HIPS_ERR_TIMEOUT = -5
 HIPS_ERR_TOO_LARGE = -6
+HIPS_ERR_INTERNAL = -7
+MAX_STAGES = 8
 NOALLOC_SCRATCH_BYTES = 512 << 10
 
 HIPS_F32 = 0
@@ -42,6 +44,13 @@ class HipsError(RuntimeError):
         super().__init__(f"{fn} failed: {code} ({detail})")
 
 
+class Stage(ctypes.Structure):
+    """Mirror of ``hips_stage`` (include/hip_sparse.h): one pruning stage."""
+
+    _fields_ = [("chunk_size", ctypes.c_int32), ("stage_k", ctypes.c_int32),
+                ("stride_q", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 class Params(ctypes.Structure):
     """Mirror of ``hips_params`` (include/hip_sparse.h)."""
 
@@ -56,6 +65,8 @@ class Params(ctypes.Structure):
         ("window", ctypes.c_int32), ("flags", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
+        ("n_stages", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("stages", ctypes.POINTER(Stage)),
     ]
 
 
@@ -115,13 +126,25 @@ def _check(fn: str, code: int) -> None:
 
 def params(*, batch, n_qheads, n_kvheads, seq_len, q_len, q_pos0, dtype, block_q=1, block_k=1,
            topk=1, sink=0, window=0, mask_len=None, kv_capacity=None, head_dim=128,
-           workspace=0, workspace_bytes=0, stream=0, flags=0) -> Params:
-    return Params(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, head_dim=head_dim,
-                  seq_len=seq_len, mask_len=seq_len if mask_len is None else mask_len,
-                  kv_capacity=seq_len if kv_capacity is None else kv_capacity, q_len=q_len,
-                  dtype=dtype, q_pos0=q_pos0, block_q=block_q, block_k=block_k, topk=topk,
-                  sink=sink, window=window, flags=flags, workspace=workspace or None,
-                  workspace_bytes=workspace_bytes, stream=stream or None)
+           workspace=0, workspace_bytes=0, stream=0, flags=0, stages=()) -> Params:
+    """stages: (chunk_size, stage_k, stride_q) per pruning stage (stage_k 0
+    keeps every chunk); topk is then the iteration's budget."""
+    p = Params(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, head_dim=head_dim,
+               seq_len=seq_len, mask_len=seq_len if mask_len is None else mask_len,
+               kv_capacity=seq_len if kv_capacity is None else kv_capacity, q_len=q_len,
+               dtype=dtype, q_pos0=q_pos0, block_q=block_q, block_k=block_k, topk=topk,
+               sink=sink, window=window, flags=flags, workspace=workspace or None,
+               workspace_bytes=workspace_bytes, stream=stream or None)
+    set_stages(p, stages)
+    return p
+
+
+def set_stages(p: Params, stages) -> None:
+    """Point p at a stage list (kept alive with p)."""
+    arr = (Stage * max(1, len(stages)))(*[Stage(int(c), int(k), int(r), 0) for c, k, r in stages])
+    p._stage_array = arr
+    p.n_stages = len(stages)
+    p.stages = ctypes.cast(arr, ctypes.POINTER(Stage)) if stages else None
 
 
 def idx_row_stride(p: Params) -> int:
@@ -228,14 +251,14 @@ class Session:
 
     def __init__(self, *, batch, n_qheads, n_kvheads, seq_len, q_len, q_pos0, dtype, block_q=1,
                  block_k=1, topk=1, sink=0, window=0, mask_len=None, kv_capacity=None,
-                 stream=None, flags=0):
+                 stream=None, flags=0, stages=()):
         import torch
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.p = params(batch=batch, n_qheads=n_qheads, n_kvheads=n_kvheads, seq_len=seq_len,
                         q_len=q_len, q_pos0=q_pos0, dtype=dtype, block_q=block_q,
                         block_k=block_k, topk=topk, sink=sink, window=window,
                         mask_len=mask_len, kv_capacity=kv_capacity,
-                        stream=self.stream.cuda_stream, flags=flags)
+                        stream=self.stream.cuda_stream, flags=flags, stages=stages)
         need = max(workspace_size(self.p, op) for op in (OP_MASK, OP_SPARSE, OP_DENSE, OP_MASK_SPARSE))
         if need == 0:
             raise HipsError("hip_workspace_size", HIPS_ERR_INVALID_ARG, "invalid parameters")

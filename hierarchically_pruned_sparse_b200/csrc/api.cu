@@ -49,6 +49,18 @@ int validate(const hips_params* p, int op) {
   }
   const double elems = static_cast<double>(p->batch) * p->n_kvheads * p->kv_capacity * p->head_dim;
   if (elems > 4.0e18) return HIPS_ERR_INVALID_ARG;
+  if (op == HIPS_OP_MASK || op == HIPS_OP_MASK_SPARSE) {
+    // pruning stages (struct hips_stage): sizes in whole blocks, each
+    // dividing the one before, kept keys in whole chunks
+    if (p->n_stages < 0 || p->n_stages > HIPS_MAX_STAGES) return HIPS_ERR_INVALID_ARG;
+    if (p->n_stages > 0 && !p->stages) return HIPS_ERR_INVALID_ARG;
+    for (int i = 0; i < p->n_stages; ++i) {
+      const hips_stage& g = p->stages[i];
+      if (g.chunk_size <= 0 || g.chunk_size % p->block_k || g.stride_q < 1) return HIPS_ERR_INVALID_ARG;
+      if (g.stage_k < 0 || g.stage_k % g.chunk_size) return HIPS_ERR_INVALID_ARG;
+      if (i > 0 && p->stages[i - 1].chunk_size % g.chunk_size) return HIPS_ERR_INVALID_ARG;
+    }
+  }
   return HIPS_OK;
 }
 
@@ -72,10 +84,32 @@ int group_rows(const hips_params* p, int block_q) {
 
 // ---------------------------------------------------------------- mask plan
 
+// The pruning stages of a mask call (struct hips_stage): one step per stage
+// that ranks (stage_k > 0), each a scoring launch and a selection launch
+// per mask row; with no ranking stage, one selection step that only cuts and
+// halves. The last step writes the iteration's initial chunk lists.
+struct StageStep {
+  int c_in;     // > 0: the input is the tiling of [0, N) by c_in blocks; 0: the previous list
+  int keep;     // chunks a row keeps (0: all, nothing scored)
+  int stride_q;
+  int c_out;    // blocks per output piece
+  bool final_list;
+};
+
+struct StagePlan {
+  int nsteps;
+  StageStep steps[HIPS_MAX_STAGES + 1];
+  int cap;          // entries of a list (and scores per row)
+  int64_t lstride;  // int32 per row of a list
+  size_t bytes;     // scores, then two lists, each 256-byte aligned
+};
+
 struct MaskPlan {
   hips::MaskArgs a;
   int smem;
   size_t ws;
+  StagePlan stp;
+  size_t st_off;  // workspace offset of the stage buffers
   bool mma;  // tensor-core kernel (bf16 or e5m2 keys) or CUDA-core kernel
   bool norms;  // key-block norm pre-pass into the workspace (many-row masks)
   bool decode;  // the decode kernel (one query position per mask row)
@@ -152,7 +186,7 @@ int plan_mask_mma(const hips_params* p, int cluster_cap, MaskPlan* plan) {
   return HIPS_OK;
 }
 
-int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan, bool attend = false) {
+int plan_mask_kernel(const hips_params* p, int cluster_cap, MaskPlan* plan, bool attend) {
   hips::MaskArgs& a = plan->a;
   a = hips::MaskArgs{};
   plan->decode = false;
@@ -204,6 +238,72 @@ int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan, bool attend
   }
   if (plan->smem > kMaxSmem) return HIPS_ERR_UNSUPPORTED;
   plan->ws = kStatusBytes;
+  return HIPS_OK;
+}
+
+// Steps and buffers of the pruning stages, with bounds taken over every mask
+// row: the first ranking stage has at most ceil(N / c) chunks, a later one at
+// most (the chunks kept before) x (their size / its size), each at most
+// kStageMaxChunks; the iteration must start from at most n0max chunks.
+int plan_stages(const hips_params* p, int64_t units, StagePlan* sp) {
+  sp->nsteps = 0;
+  sp->bytes = 0;
+  sp->cap = 0;
+  sp->lstride = 0;
+  if (p->n_stages == 0) return HIPS_OK;
+  const int64_t bk = p->block_k;
+  const int64_t nmax = cdiv(std::min<int64_t>(p->q_pos0 + p->q_len, p->seq_len), bk);
+  const int64_t n0max = p->topk / bk;
+  const hips_stage* st = p->stages;
+  const int S = p->n_stages;
+  int ranked[HIPS_MAX_STAGES];
+  int nr = 0;
+  for (int i = 0; i < S; ++i)
+    if (st[i].stage_k > 0) ranked[nr++] = i;
+  const int64_t c_last = st[S - 1].chunk_size / bk;
+  int64_t cap = n0max, kept = 0, kept_c = 1;
+  for (int t = 0; t < nr; ++t) {
+    const hips_stage& g = st[ranked[t]];
+    const int64_t c = g.chunk_size / bk;
+    const int64_t cands = t == 0 ? cdiv(nmax, c) : kept * (kept_c / c);
+    const int64_t keep = g.stage_k / g.chunk_size;
+    if (cands > hips::kStageMaxChunks) return HIPS_ERR_UNSUPPORTED;
+    cap = std::max(cap, cands);
+    StageStep& step = sp->steps[sp->nsteps++];
+    step.c_in = t == 0 ? static_cast<int>(c) : 0;
+    step.keep = static_cast<int>(std::min<int64_t>(keep, 1 << 30));
+    step.stride_q = g.stride_q;
+    step.final_list = t + 1 == nr;
+    step.c_out = static_cast<int>(step.final_list ? c_last : st[ranked[t + 1]].chunk_size / bk);
+    kept = std::min(keep, cands);
+    kept_c = c;
+  }
+  int64_t pieces;
+  if (nr == 0) {
+    StageStep& step = sp->steps[sp->nsteps++];
+    step = StageStep{static_cast<int>(c_last), 0, 1, static_cast<int>(c_last), true};
+    pieces = cdiv(nmax, c_last);
+  } else {
+    pieces = kept * (kept_c / c_last);
+  }
+  if (pieces > n0max) return HIPS_ERR_UNSUPPORTED;
+  cap = std::max(cap, pieces);
+  if (cap > (int64_t{1} << 22)) return HIPS_ERR_UNSUPPORTED;
+  sp->cap = static_cast<int>(cap);
+  sp->lstride = 4 + 2 * cap;
+  const size_t scores = (static_cast<size_t>(units) * cap * sizeof(float) + 255) / 256 * 256;
+  const size_t list = (static_cast<size_t>(units) * sp->lstride * sizeof(int32_t) + 255) / 256 * 256;
+  sp->bytes = scores + 2 * list;
+  return HIPS_OK;
+}
+
+int plan_mask(const hips_params* p, int cluster_cap, MaskPlan* plan, bool attend = false) {
+  int st = plan_mask_kernel(p, cluster_cap, plan, attend);
+  if (st) return st;
+  st = plan_stages(p, plan->a.units, &plan->stp);
+  if (st) return st;
+  plan->st_off = (plan->ws + 255) / 256 * 256;
+  if (plan->stp.nsteps) plan->ws = plan->st_off + plan->stp.bytes;
   return HIPS_OK;
 }
 
@@ -366,6 +466,64 @@ bool fusable(const MaskPlan& plan) {
                          plan.a.rows_max <= hips::mask_mma_fused_rows());
 }
 
+// Launch the pruning stages of a mask call; *init gets the list the
+// iteration starts from.
+int run_stages(const void* q, const void* k, const hips_params* p, const MaskPlan& plan,
+               cudaStream_t stream, const int32_t** init) {
+  const StagePlan& sp = plan.stp;
+  const hips::MaskArgs& m = plan.a;
+  unsigned char* base = static_cast<unsigned char*>(p->workspace) + plan.st_off;
+  const size_t scores = (static_cast<size_t>(m.units) * sp.cap * sizeof(float) + 255) / 256 * 256;
+  const size_t list = (static_cast<size_t>(m.units) * sp.lstride * sizeof(int32_t) + 255) / 256 * 256;
+  int32_t* lists[2] = {reinterpret_cast<int32_t*>(base + scores),
+                       reinterpret_cast<int32_t*>(base + scores + list)};
+  hips::StageArgs s{};
+  s.q = q;
+  s.k = k;
+  s.status = static_cast<hips::Status*>(p->workspace);
+  s.dtype = m.dtype;
+  s.n_qheads = m.n_qheads;
+  s.n_mheads = m.n_kvheads;
+  s.group = m.group;
+  s.kv_heads = m.kv_heads;
+  s.kv_div = m.kv_div;
+  s.q_len = m.q_len;
+  s.block_q = m.block_q;
+  s.block_k = m.block_k;
+  s.nqb = m.nqb;
+  s.n0max = m.n0max;
+  s.units = m.units;
+  s.seq_len = m.seq_len;
+  s.kv_cap = m.kv_cap;
+  s.q_pos0 = m.q_pos0;
+  s.lstride = sp.lstride;
+  s.cap = sp.cap;
+  s.scores = reinterpret_cast<float*>(base);
+  // one wave of scoring CTAs (one per SM; each keeps 32 groups' key rows
+  // in flight), at least 32 chunks each
+  s.slices = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(kPlanSMs / m.units, cdiv(sp.cap, 32))));
+  for (int i = 0; i < sp.nsteps; ++i) {
+    const StageStep& step = sp.steps[i];
+    s.c_in = step.c_in;
+    s.c_list = i ? sp.steps[i - 1].c_out : step.c_in;
+    s.in = i ? lists[(i - 1) & 1] : nullptr;
+    s.out = lists[i & 1];
+    s.keep = step.keep;
+    s.stride_q = step.stride_q;
+    s.c_out = step.c_out;
+    s.final_list = step.final_list ? 1 : 0;
+    if (step.keep > 0) {
+      const cudaError_t e = hips::launch_stage_score(s, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+    const cudaError_t e = hips::launch_stage_select(s, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  *init = lists[(sp.nsteps - 1) & 1];
+  return HIPS_OK;
+}
+
 // Plan and launch the mask kernel (with the fused attention when v and out
 // are given). A cluster of C CTAs needs C free SMs of one GPC: take the
 // largest cluster for which every mask row is resident at once (one wave);
@@ -379,6 +537,11 @@ int launch_mask(const void* q, const void* k, const hips_params* params, int32_t
   st = check_workspace(params, plan.ws);
   if (st) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(params->stream);
+  const int32_t* init = nullptr;
+  if (plan.stp.nsteps) {
+    st = run_stages(q, k, params, plan, stream, &init);
+    if (st) return st;
+  }
   for (int cap = 16; cap >= 1; cap = std::min(cap - 1, plan.a.cluster - 1)) {
     st = plan_mask(params, cap, &plan, attend);
     if (st) return st;
@@ -390,6 +553,11 @@ int launch_mask(const void* q, const void* k, const hips_params* params, int32_t
     hips::MaskArgs& a = plan.a;
     a.q = q; a.k = k; a.idx = idx_out;
     a.status = static_cast<hips::Status*>(params->workspace);
+    if (init) {
+      a.init = init;
+      a.init_stride = plan.stp.lstride;
+      a.init_cap = plan.stp.cap;
+    }
     if (plan.norms) {
       a.knorm = reinterpret_cast<const float*>(static_cast<unsigned char*>(params->workspace) + kStatusBytes);
       const cudaError_t e = hips::launch_key_block_norms(a, params->batch, stream);
@@ -486,7 +654,7 @@ int hip_check_status(const hips_params* params) {
   if (host.flags == 0) return HIPS_OK;
   st = cuda_status(cudaMemset(params->workspace, 0, kStatusBytes));
   if (st) return st;
-  return HIPS_ERR_TIMEOUT;
+  return (host.flags & hips::kStatusTimeout) ? HIPS_ERR_TIMEOUT : HIPS_ERR_INTERNAL;
 }
 
 int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* idx_out) {
@@ -536,6 +704,7 @@ const char* hip_error_string(int status) {
     case HIPS_ERR_CUDA: return "CUDA launch failed";
     case HIPS_ERR_TIMEOUT: return "a bounded device wait expired";
     case HIPS_ERR_TOO_LARGE: return "request exceeds the library's built-in scratch size";
+    case HIPS_ERR_INTERNAL: return "a device-side bound check failed";
     default: return "unknown status";
   }
 }

@@ -64,36 +64,6 @@ constexpr int kBuckets = 2048;
 constexpr int kPS = kD + 4;      // partial row: m, l, pad, pad, o[128]
 constexpr int kStashMax = 32768; // bytes of last-round dots kept for the attention
 
-// A lane's share of one key (or value) row in the canonical order: slices
-// l8 and l8 + 8 (elements 8 l8 .. 8 l8 + 7 and 64 + 8 l8 .. 64 + 8 l8 + 7),
-// held raw in registers until used (loaded from a row staged in shared
-// memory).
-template <typename KvT>
-struct Lane16;
-
-template <>
-struct Lane16<uint8_t> {  // fp8 e5m2 codes, widened exactly
-  uint2 a, b;
-  __device__ __forceinline__ void load_smem(const unsigned char* row, int l8) {
-    a = *reinterpret_cast<const uint2*>(row + l8 * 8);
-    b = *reinterpret_cast<const uint2*>(row + 64 + l8 * 8);
-  }
-  __device__ __forceinline__ void zero() { a = b = make_uint2(0, 0); }
-  __device__ __forceinline__ void get(float (&x)[16]) const {
-    e5m2x4_to_f32(a.x, x);
-    e5m2x4_to_f32(a.y, x + 4);
-    e5m2x4_to_f32(b.x, x + 8);
-    e5m2x4_to_f32(b.y, x + 12);
-  }
-};
-
-// Keys a group requests before using the first (register budget: the query
-// rows take 16 RC floats per lane).
-template <typename KvT, int RC>
-__host__ __device__ constexpr int keys_per_batch() {
-  return std::is_same<KvT, float>::value ? (RC <= 4 ? 4 : 1) : (RC <= 4 ? 8 : 2);
-}
-
 __device__ __forceinline__ void cluster_arrive_release() {
   asm volatile("barrier.cluster.arrive.release;" ::: "memory");
 }
@@ -192,7 +162,12 @@ __global__ void __launch_bounds__(kT, 1) decode_kernel(MaskArgs a) {
   const int bk = a.block_k;
   const int lbk = __ffs(bk) - 1;
   const int N_blocks = (Tc + bk - 1) / bk;
-  const int n0 = min(a.n0max, N_blocks);
+  // initial chunks: n0 uniform ones, or the list the pruning stages left
+  // (then every round keeps its n_keep entry)
+  const int32_t* init = a.init ? a.init + unit * a.init_stride : nullptr;
+  const int n_unif = min(a.n0max, N_blocks);
+  const int n_init = init ? init[0] : n_unif;
+  const int n0 = init ? init[1] : n_unif;
   const int per_cta = a.per_cta;
   const int nbuf = (2 * a.n0max + 15) & ~15;
   const bool attend = a.out != nullptr;
@@ -292,28 +267,36 @@ __global__ void __launch_bounds__(kT, 1) decode_kernel(MaskArgs a) {
   const int sw0 = min(nsw, rank * sw_per), sw1 = min(nsw, sw0 + sw_per);
   auto sw_block = [&](int e) -> int { return e < lead ? e : cutb + (e - lead); };
   for (int i = tid; i < kBuckets; i += kT) hist[i] = 0;
-  // ---- round-1 candidates: the halves of the n0 chunks [iN/n0, (i+1)N/n0)
-  // (a one-block chunk stays whole); thread t owns chunks [t pc, (t+1) pc)
+  // ---- round-1 candidates: the halves of the n_init initial chunks, the
+  // uniform [iN/n0, (i+1)N/n0) or the stages' list (a one-block chunk stays
+  // whole); thread t owns chunks [t pc, (t+1) pc)
   int ncand, nlong;
   {
-    const int pc = (n0 + kT - 1) / kT;
-    const int lo = min(n0, tid * pc), hi = min(n0, lo + pc);
-    auto bound = [&](int i) -> int {
-      return static_cast<int>(static_cast<int64_t>(i) * N_blocks / n0);
+    const int pc = (n_init + kT - 1) / kT;
+    const int lo = min(n_init, tid * pc), hi = min(n_init, lo + pc);
+    auto chunk_at = [&](int i, int& s0, int& e0) {
+      if (init) {
+        s0 = init[4 + i];
+        e0 = init[4 + a.init_cap + i];
+      } else {
+        s0 = static_cast<int>(static_cast<int64_t>(i) * N_blocks / n_unif);
+        e0 = static_cast<int>(static_cast<int64_t>(i + 1) * N_blocks / n_unif);
+      }
     };
     int cnt = 0, nl = 0;
-    for (int i = lo, s0 = bound(lo); i < hi; ++i) {
-      const int e0 = bound(i + 1);
+    for (int i = lo; i < hi; ++i) {
+      int s0, e0;
+      chunk_at(i, s0, e0);
       cnt += e0 - s0 > 1 ? 2 : 1;
       nl += e0 - s0 > 1 ? 1 : 0;
-      s0 = e0;
     }
     int tot;
     int pos = block_excl_scan(cnt | (nl << 16), scratch, tot) & 0xffff;
     ncand = tot & 0xffff;
     nlong = tot >> 16;
-    for (int i = lo, s0 = bound(lo); i < hi; ++i) {
-      const int e0 = bound(i + 1);
+    for (int i = lo; i < hi; ++i) {
+      int s0, e0;
+      chunk_at(i, s0, e0);
       if (e0 - s0 > 1) {
         const int m = s0 + (e0 - s0) / 2;
         cs_all[pos] = s0; ce_all[pos] = m; ++pos;
@@ -321,7 +304,6 @@ __global__ void __launch_bounds__(kT, 1) decode_kernel(MaskArgs a) {
       } else {
         cs_all[pos] = s0; ce_all[pos] = e0; ++pos;
       }
-      s0 = e0;
     }
   }
   __syncthreads();
@@ -404,8 +386,8 @@ __global__ void __launch_bounds__(kT, 1) decode_kernel(MaskArgs a) {
             const int kq = k0 + u;
             const int i = gi + kG * (kq >> lbk);  // candidate of the batch
             const int kt = kq & (bk - 1);
-            Lane16<KvT> kr;
-            if (kq < nk) kr.load_smem(slot + (i * bk + kt) * kRowB, l8);
+            Row16<KvT> kr;
+            if (kq < nk) kr.load(slot + (i * bk + kt) * kRowB, l8);
             else kr.zero();
             float x[16];
             kr.get(x);
@@ -808,8 +790,8 @@ __global__ void __launch_bounds__(kT, 1) decode_kernel(MaskArgs a) {
           float s2[RC];
 #pragma unroll
           for (int r = 0; r < RC; ++r) s2[r] = r < R ? st[r] * sl2 : -INFINITY;
-          Lane16<KvT> vr;
-          vr.load_smem(slot + ((item - p0) * bk + kt) * kRowB, l8);
+          Row16<KvT> vr;
+          vr.load(slot + ((item - p0) * bk + kt) * kRowB, l8);
           float vx[16];
           vr.get(vx);
           accumulate(s2, vx);
@@ -828,10 +810,10 @@ __global__ void __launch_bounds__(kT, 1) decode_kernel(MaskArgs a) {
           const int item = inb ? kq >> lbk : 0, kt = kq & (bk - 1);
           const bool ok = inb && kt < rows_at(b_block(j0 + item));
           const unsigned char* kblk = slot + (b0 - p0 + 2 * item) * blk_bytes;
-          Lane16<KvT> kr, vr;
+          Row16<KvT> kr, vr;
           if (ok) {
-            kr.load_smem(kblk + kt * kRowB, l8);
-            vr.load_smem(kblk + blk_bytes + kt * kRowB, l8);
+            kr.load(kblk + kt * kRowB, l8);
+            vr.load(kblk + blk_bytes + kt * kRowB, l8);
           } else {
             kr.zero();
             vr.zero();

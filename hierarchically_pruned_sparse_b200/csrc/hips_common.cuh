@@ -11,7 +11,8 @@ constexpr int kThreads = 256;      // threads of the CUDA-core kernels
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxN0 = 2048;       // topk / block_k
 constexpr int kMaxDevices = 64;
-constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusTimeout = 1u;  // a bounded wait gave up
+constexpr unsigned kStatusBound = 2u;    // a list outgrew its planned capacity
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 // values of enum hips_dtype (include/hip_sparse.h)
 constexpr int kDtypeF32 = 0, kDtypeBf16 = 1, kDtypeBf16E5m2 = 2;
@@ -216,6 +217,63 @@ __device__ __forceinline__ void load_row16<uint8_t>(const unsigned char* row, in
 
 template <typename T>
 constexpr int row_bytes() { return kD * static_cast<int>(sizeof(T)); }
+
+// A lane's share of one key (or value) row in the canonical order, held raw
+// in registers until used: slices l8 and l8 + 8 (elements 8 l8 .. 8 l8 + 7
+// and 64 + 8 l8 .. 64 + 8 l8 + 7). load() takes a global or a shared-memory
+// row (generic addressing); get() widens to fp32 (exactly, for every type).
+template <typename KvT>
+struct Row16;
+
+template <>
+struct Row16<uint16_t> {  // bf16
+  uint4 a, b;
+  __device__ __forceinline__ void load(const unsigned char* row, int l8) {
+    a = *reinterpret_cast<const uint4*>(row + l8 * 16);
+    b = *reinterpret_cast<const uint4*>(row + 128 + l8 * 16);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void get(float (&x)[16]) const {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[2 * i] = bf16lo(w[i]);
+      x[2 * i + 1] = bf16hi(w[i]);
+    }
+  }
+};
+
+template <>
+struct Row16<float> {
+  float4 a0, a1, b0, b1;
+  __device__ __forceinline__ void load(const unsigned char* row, int l8) {
+    const float4* p = reinterpret_cast<const float4*>(row + l8 * 32);
+    const float4* q = reinterpret_cast<const float4*>(row + 256 + l8 * 32);
+    a0 = p[0]; a1 = p[1]; b0 = q[0]; b1 = q[1];
+  }
+  __device__ __forceinline__ void zero() { a0 = a1 = b0 = b1 = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void get(float (&x)[16]) const {
+    x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w; x[4] = a1.x; x[5] = a1.y; x[6] = a1.z;
+    x[7] = a1.w; x[8] = b0.x; x[9] = b0.y; x[10] = b0.z; x[11] = b0.w; x[12] = b1.x;
+    x[13] = b1.y; x[14] = b1.z; x[15] = b1.w;
+  }
+};
+
+template <>
+struct Row16<uint8_t> {  // fp8 e5m2 codes, widened exactly
+  uint2 a, b;
+  __device__ __forceinline__ void load(const unsigned char* row, int l8) {
+    a = *reinterpret_cast<const uint2*>(row + l8 * 8);
+    b = *reinterpret_cast<const uint2*>(row + 64 + l8 * 8);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_uint2(0, 0); }
+  __device__ __forceinline__ void get(float (&x)[16]) const {
+    e5m2x4_to_f32(a.x, x);
+    e5m2x4_to_f32(a.y, x + 4);
+    e5m2x4_to_f32(b.x, x + 8);
+    e5m2x4_to_f32(b.y, x + 12);
+  }
+};
 
 // Canonical-order reduction of RC lane partials over the 8 lanes of a group:
 // level 1 adds lanes (l, l^4), level 2 (l, l^2), level 3 (l, l^1), i.e.

@@ -47,6 +47,40 @@ struct MaskArgs {
   int stash_dots;
   int slot_bytes;
   int list_cap;  // entries of its staging list
+  // pruning stages ran before: the initial chunks of unit u are the list at
+  // init + u * init_stride ([count, n_keep, 0, 0, starts[init_cap],
+  // ends[init_cap]]) instead of the n0 uniform chunks; n_keep replaces n0
+  const int32_t* init;
+  int64_t init_stride;
+  int init_cap;
+};
+
+// One step of the pruning stages (stages.cu): the chunks of every mask row
+// -- the tiling of [0, N) in chunks of c_in blocks (c_in > 0), or the list
+// `in` -- are scored (stage_score) and the best `keep` of them (all when
+// keep is 0) are cut into pieces of c_out blocks and written to `out`
+// (stage_select). With final_list the pieces are then halved for as long as
+// the halves number at most n0, the result being the iteration's initial
+// chunks. Lists hold per unit lstride int32: [count, n_keep, 0, 0,
+// starts[cap], ends[cap]] (n_keep only in a final list).
+struct StageArgs {
+  const void* q;
+  const void* k;
+  Status* status;
+  int dtype, n_qheads, n_mheads, group, kv_heads, kv_div, q_len, block_q, block_k, nqb, n0max;
+  int64_t units, seq_len, kv_cap, q_pos0;
+  int c_in;
+  int c_list;  // blocks of every input chunk but the last (c_in, or the previous step's c_out)
+  const int32_t* in;
+  int32_t* out;
+  int64_t lstride;
+  int cap;
+  float* scores;  // per unit cap floats
+  int keep;
+  int stride_q;
+  int c_out;
+  int final_list;
+  int slices;  // CTAs per unit of the scoring launch
 };
 
 struct AttnArgs {
@@ -92,6 +126,13 @@ int decode_max_rows();
 int decode_smem_bytes(MaskArgs& a, bool attend, int smem_cap);
 int decode_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_decode(const MaskArgs& a, int smem, cudaStream_t stream);
+
+// Pruning stages (stages.cu). A stage of a mask row ranks at most
+// kStageMaxChunks chunks (the selection keeps their score keys in shared
+// memory).
+constexpr int kStageMaxChunks = 36864;
+cudaError_t launch_stage_score(const StageArgs& a, cudaStream_t stream);
+cudaError_t launch_stage_select(const StageArgs& a, cudaStream_t stream);
 
 // Tensor-core attention for query blocks, bf16 (attn_mma.cu)
 int attn_mma_smem_bytes(int table_items);

@@ -99,7 +99,12 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
   const int64_t Tc = min64(q_last + 1, a.seq_len);
   const int bk = a.block_k;
   const int64_t N = (Tc + bk - 1) / bk;
-  const int n0 = static_cast<int>(min64(a.n0max, N));
+  // initial chunks: n0 uniform ones, or the list the pruning stages left
+  // (then every round keeps its n_keep entry)
+  const int32_t* init = a.init ? a.init + unit * a.init_stride : nullptr;
+  const int n_unif = static_cast<int>(min64(a.n0max, N));
+  const int n0 = init ? init[1] : n_unif;
+  int nch = init ? init[0] : n_unif;  // chunks in the list
   const int per_cta = a.per_cta;
 
   const MaskSmem L = mask_smem_layout(a.n0max, a.rows_pad, per_cta, C, stages);
@@ -138,10 +143,15 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
     }
     qs[e] = x;
   }
-  // step 1: n0 chunks that tile [0, N)
-  for (int i = tid; i < n0; i += kThreads) {
-    chunk_s[i] = static_cast<int>(static_cast<int64_t>(i) * N / n0);
-    chunk_e[i] = static_cast<int>(static_cast<int64_t>(i + 1) * N / n0);
+  // step 1: n0 chunks that tile [0, N) (or the stages' list)
+  for (int i = tid; i < nch; i += kThreads) {
+    if (init) {
+      chunk_s[i] = init[4 + i];
+      chunk_e[i] = init[4 + a.init_cap + i];
+    } else {
+      chunk_s[i] = static_cast<int>(static_cast<int64_t>(i) * N / n_unif);
+      chunk_e[i] = static_cast<int>(static_cast<int64_t>(i + 1) * N / n_unif);
+    }
   }
   for (int i = tid; i < kBuckets; i += kThreads) hist[i] = 0;
   __syncthreads();
@@ -175,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
 
   for (;;) {
     // ---- step 2: candidates (halves of every chunk; a 1-block chunk stays whole)
-    const int per_t = (n0 + kThreads - 1) / kThreads;
-    const int lo_t = min(n0, tid * per_t), hi_t = min(n0, lo_t + per_t);
+    const int per_t = (nch + kThreads - 1) / kThreads;
+    const int lo_t = min(nch, tid * per_t), hi_t = min(nch, lo_t + per_t);
     int cnt = 0, nlong = 0;
     for (int i = lo_t; i < hi_t; ++i) {
       const int len = chunk_e[i] - chunk_s[i];
@@ -417,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_fma_kernel(MaskArgs a) {
     }
     int total;
     int dst = block_excl_scan(nk, scratch, total);
+    nch = total;  // n0
     for (int i = lo_c; i < hi_c; ++i) {
       const int bi = bkt[i];
       if (bi > cut || (bi == cut && keep[i])) {

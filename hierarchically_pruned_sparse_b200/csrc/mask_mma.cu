@@ -346,7 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
   const int bk = a.block_k;
   const int lbk = __ffs(bk) - 1;
   const int64_t N_blocks = (Tc + bk - 1) / bk;
-  const int n0 = static_cast<int>(min64(a.n0max, N_blocks));
+  // initial chunks: n0 uniform ones, or the list the pruning stages left
+  // (then every round keeps its n_keep entry)
+  const int32_t* init = a.init ? a.init + unit * a.init_stride : nullptr;
+  const int n_unif = static_cast<int>(min64(a.n0max, N_blocks));
+  const int n_init = init ? init[0] : n_unif;
+  const int n0 = init ? init[1] : n_unif;
   const int per_cta = a.per_cta;
   const int nbuf = (2 * a.n0max + 3) & ~3;  // stride between the two candidate buffers
 
@@ -443,16 +448,25 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     if (lane == 0) qn[r] = r < R ? sqrtf(s) * kNormUp : 0.0f;
   }
 
-  // ---- candidates of round 1: the halves of the n0 initial chunks
+  // ---- candidates of round 1: the halves of the n_init initial chunks
   // (a one-block chunk stays whole); thread t owns chunks [t*pc, (t+1)*pc)
   int ncand, nlong;
   {
-    const int pc = (n0 + kThreads - 1) / kThreads;
-    const int lo = min(n0, tid * pc), hi = min(n0, lo + pc);
+    auto chunk_at = [&](int i, int& s0, int& e0) {
+      if (init) {
+        s0 = init[4 + i];
+        e0 = init[4 + a.init_cap + i];
+      } else {
+        s0 = static_cast<int>(static_cast<int64_t>(i) * N_blocks / n_unif);
+        e0 = static_cast<int>(static_cast<int64_t>(i + 1) * N_blocks / n_unif);
+      }
+    };
+    const int pc = (n_init + kThreads - 1) / kThreads;
+    const int lo = min(n_init, tid * pc), hi = min(n_init, lo + pc);
     int cnt = 0, nl = 0;
     for (int i = lo; i < hi; ++i) {
-      const int64_t s0 = static_cast<int64_t>(i) * N_blocks / n0;
-      const int64_t e0 = static_cast<int64_t>(i + 1) * N_blocks / n0;
+      int s0, e0;
+      chunk_at(i, s0, e0);
       cnt += e0 - s0 > 1 ? 2 : 1;
       nl += e0 - s0 > 1 ? 1 : 0;
     }
@@ -461,8 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_mma_kernel(MaskArgs a) {
     ncand = tot & 0xffff;
     nlong = tot >> 16;
     for (int i = lo; i < hi; ++i) {
-      const int s0 = static_cast<int>(static_cast<int64_t>(i) * N_blocks / n0);
-      const int e0 = static_cast<int>(static_cast<int64_t>(i + 1) * N_blocks / n0);
+      int s0, e0;
+      chunk_at(i, s0, e0);
       auto put = [&](int s, int e) {
         cs_all[pos] = s;
         ce_all[pos] = e;

@@ -77,7 +77,8 @@ enum hips_status {
   HIPS_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or too small */
   HIPS_ERR_CUDA = -4,        /* a CUDA launch failed */
   HIPS_ERR_TIMEOUT = -5,     /* a bounded device wait expired (from hip_check_status) */
-  HIPS_ERR_TOO_LARGE = -6    /* more scratch than hip_sparse_attn_noalloc's fixed array */
+  HIPS_ERR_TOO_LARGE = -6,   /* more scratch than hip_sparse_attn_noalloc's fixed array */
+  HIPS_ERR_INTERNAL = -7     /* a device-side bound check failed (from hip_check_status) */
 };
 
 /* Element types. HIPS_BF16_E5M2 is an fp8 KV cache: k and v hold fp8 e5m2
@@ -106,6 +107,37 @@ enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2, HIPS_OP_
  *   ignore it. */
 enum hips_flags { HIPS_FLAG_HEAD_MASKS = 1 };
 
+/* One InfiniteHiP pruning stage (the stages of the serving command's
+ * --hip-attention-config in "[Feature] Support Efficient Sparse HiP Attention
+ * (InfiniteHiP)"; Author Rebuttal to the Reviewer T2wK, Q1: the user sets per
+ * iteration how many chunks are kept, how chunks are broken down and how
+ * their representatives are picked). Stage 1 cuts the key blocks [0, N) of a
+ * mask row into chunks of chunk_size keys aligned at multiples of it (the
+ * last one clipped); a later stage cuts every chunk kept by the one before
+ * into pieces of its own size. A stage with stage_k > 0 scores each chunk
+ * [s, e) (in blocks) by its centre block s + (e - s) / 2 -- the max over
+ * the stage's query rows and the block's keys they see of q.k -- and keeps
+ * the stage_k / chunk_size best by (score desc, start asc); stage_k = 0 (null
+ * on the page) keeps every chunk. The stage's query rows are the mask's
+ * query heads at the positions i1-1, i1-1-stride_q, ... of the query block
+ * [i0, i1) (the block's last row, which sees every key of the range, always
+ * scores). After the stages the hierarchical iteration (hip_mask) runs with
+ * k = topk (the page's second_stage_k) from the surviving chunks instead of
+ * topk / block_k uniform ones: every round halves each chunk and keeps the
+ * topk / block_k best halves (all of them while there are no more). The
+ * page's stage_block_size_q is the mask's block_q; its stage_stride (1 in
+ * every stage of the page's configuration) has no field. */
+typedef struct hips_stage {
+  int32_t chunk_size;  /* keys per chunk: a multiple of block_k that divides the
+                          previous stage's chunk_size */
+  int32_t stage_k;     /* keys kept: a multiple of chunk_size; 0 keeps every chunk */
+  int32_t stride_q;    /* query-row stride of the stage's scoring, >= 1 */
+  int32_t reserved;    /* 0 */
+} hips_stage;
+
+/* Most stages of one schedule. */
+#define HIPS_MAX_STAGES 8
+
 typedef struct hips_params {
   int32_t batch;      /* sequences */
   int32_t n_qheads;   /* query heads; a multiple of n_kvheads */
@@ -128,6 +160,16 @@ typedef struct hips_params {
   void* workspace;    /* device scratch, see hip_workspace_size */
   size_t workspace_bytes;
   void* stream;       /* cudaStream_t */
+  int32_t n_stages;   /* pruning stages before the iteration, 0..HIPS_MAX_STAGES */
+  int32_t reserved;   /* 0 */
+  const hips_stage* stages; /* HOST array of n_stages entries (NULL when 0),
+                          read during each call only. The mask of a schedule
+                          needs, per mask row, at most topk / block_k chunks
+                          at the last stage's size before the iteration
+                          (worst case over the rows, from the bounds that
+                          stage_k and the key range give); larger schedules
+                          return HIPS_ERR_UNSUPPORTED. Attention-only calls
+                          ignore the stages. */
 } hips_params;
 
 /* Entries of one idx row: 1 (nnz) + the largest possible nnz. */
@@ -141,13 +183,17 @@ HIPS_API size_t hip_workspace_size(const hips_params* params, int op);
 HIPS_API int hip_workspace_init(const hips_params* params);
 
 /* Synchronise params->stream, read and clear the status block. Returns
- * HIPS_OK, or HIPS_ERR_TIMEOUT if some kernel gave up a bounded wait since
- * the last check (its outputs are then undefined). */
+ * HIPS_OK, HIPS_ERR_TIMEOUT if some kernel gave up a bounded wait since the
+ * last check, or HIPS_ERR_INTERNAL if a kernel found a list longer than its
+ * planned capacity (the outputs of the calls since are then undefined). */
 HIPS_API int hip_check_status(const hips_params* params);
 
 /* Hierarchical top-k mask (see above). q: [B, Hq, q_len, d]; k: [B, Hkv,
  * kv_capacity, d]; keys [0, seq_len) are visible. idx_out: int32 [B, Hkv,
- * n_qblocks, row_stride], fully written (padding included). */
+ * n_qblocks, row_stride], fully written (padding included). With
+ * params->n_stages > 0 the pruning stages (struct hips_stage) run first, in
+ * launches of their own on params->stream, and the iteration starts from
+ * their survivors. */
 HIPS_API int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* idx_out);
 
 /* Block-sparse attention over idx (as written by hip_mask at mask_len keys)

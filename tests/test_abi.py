@@ -191,3 +191,49 @@ def test_head_masks_plan_decode_and_prefill(flags):
                       topk=512, sink=16, window=64, flags=flags)
         assert hb.workspace_size(p, hb.OP_MASK) >= 256
         assert hb.workspace_size(p, hb.OP_SPARSE) >= 256
+
+
+# ---------------------------------------------------------------- pruning stages
+# (struct hips_stage: the stages of the serving command's --hip-attention-config
+# in "[Feature] Support Efficient Sparse HiP Attention (InfiniteHiP)")
+PR_LIKE = ((128, 0, 4), (32, 32768, 4), (8, 8192, 1))
+
+
+def test_stage_schedules_are_sized_by_their_bounds():
+    plain = hb.workspace_size(_decode_params(), hb.OP_MASK)
+    staged = hb.workspace_size(_decode_params(stages=PR_LIKE), hb.OP_MASK)
+    # 8 mask rows: scores for 4096 chunks (65536 blocks in chunks of 16) and
+    # two lists of 4 + 2 x 4096 int32, each area rounded up to 256 bytes
+    cap, rows = 4096, 8
+
+    def up(n):
+        return (n + 255) // 256 * 256
+
+    assert staged == up(plain) + up(rows * cap * 4) + 2 * up(rows * (4 + 2 * cap) * 4)
+    # attention-only calls ignore the stages
+    assert hb.workspace_size(_decode_params(stages=PR_LIKE), hb.OP_SPARSE) == \
+        hb.workspace_size(_decode_params(), hb.OP_SPARSE)
+
+
+@pytest.mark.parametrize("stages", [
+    ((3, 0, 1),),                    # not a whole number of 2-key blocks
+    ((32, 48, 1),),                  # stage_k not a whole number of chunks
+    ((32, 0, 1), (128, 0, 1)),       # a chunk size that does not divide the previous one
+    ((32, 0, 0),),                   # stride 0
+    ((32, -32, 1),),                 # negative stage_k
+    tuple((2, 0, 1) for _ in range(9)),  # more than HIPS_MAX_STAGES
+])
+def test_bad_stage_schedules_are_rejected(stages):
+    p = _decode_params(stages=stages)
+    assert hb.workspace_size(p, hb.OP_MASK) == 0
+    assert hb.workspace_size(p, hb.OP_MASK_SPARSE) == 0
+    assert hb.workspace_size(p, hb.OP_SPARSE) > 0  # the attention does not read them
+
+
+def test_stage_schedules_that_leave_more_than_n0_chunks_are_unsupported():
+    # the iteration starts from at most topk / block_k = 1024 chunks: 8-key
+    # chunks that all survive (16384 of them at 128k keys) are too many, so
+    # are 2048 survivors of a stage that keeps 16384 keys in 8-key chunks
+    assert hb.workspace_size(_decode_params(stages=((8, 0, 1),)), hb.OP_MASK) == 0
+    assert hb.workspace_size(_decode_params(stages=((8, 16384, 1),)), hb.OP_MASK) == 0
+    assert hb.workspace_size(_decode_params(stages=((8, 8192, 1),)), hb.OP_MASK) > 0
