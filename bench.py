@@ -68,6 +68,9 @@ def parse():
                     help="default run: leave out the nested prefill measurement")
     ap.add_argument("--no-dense", action="store_true",
                     help="decode: leave out the dense-attention comparison")
+    ap.add_argument("--stages", default="",
+                    help="InfiniteHiP pruning stages before the mask, chunk_size:stage_k:stride_q "
+                         "per stage, comma-separated (topk is then second_stage_k)")
     return ap.parse_args()
 
 
@@ -84,6 +87,17 @@ def peaks():
 
 
 HEAD_MASKS = False  # --head-masks: one mask per query head instead of per KV-head group
+STAGES = ()  # --stages: InfiniteHiP pruning stages (chunk_size, stage_k, stride_q) before the mask
+
+
+def stage_launches() -> int:
+    """Kernel launches the stages add to a mask call: a scoring and a
+    selection launch per stage that ranks, or one selection launch when
+    none ranks."""
+    if not STAGES:
+        return 0
+    ranked = sum(1 for _, k, _ in STAGES if k > 0)
+    return 2 * ranked if ranked else 1
 
 
 def counting_view(w: W.Workload) -> W.Workload:
@@ -94,7 +108,8 @@ def counting_view(w: W.Workload) -> W.Workload:
 
 def oracle_layer_shape(w: W.Workload):
     import oracle
-    return oracle.shape(head_dim=w.head_dim, per_head=int(HEAD_MASKS), **layer_shape(w))
+    return oracle.shape(head_dim=w.head_dim, per_head=int(HEAD_MASKS), stages=STAGES,
+                        **layer_shape(w))
 
 
 def layer_shape(w: W.Workload):
@@ -472,6 +487,8 @@ def config_of(w: W.Workload, layers: int):
            "kv_cache": {"e5m2": "fp8 e5m2 (bf16 q and out)"}.get(w.dtype, w.dtype)}
     if w.kind == "decode" and w.refresh > 1:
         cfg["mask_refresh"] = w.refresh
+    if STAGES:
+        cfg["stages"] = [{"chunk_size": c, "stage_k": k or None, "stride_q": r} for c, k, r in STAGES]
     if layers:
         cfg["l2"] = (f"{layers} rotating layer buffers; the steps between two uses of a layer "
                      f"touch {layers * touched_bytes(w) / L2_BYTES:.1f}x the L2 (no flush)")
@@ -586,6 +603,7 @@ def ours_decode(args, w: W.Workload, world: int, rank: int, dev):
     # the workspace is sized at the longest cache of the reuse steps
     shp.update(seq_len=T + rm - 1, q_pos0=T + rm - 2)
     sess = hb.Session(dtype=code, flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0, stream=stream,
+                      stages=STAGES,
                       mask_len=T, **shp)
     sess.set(seq_len=T, q_pos0=T - 1)
     lay.idxs = [sess.new_idx() for _ in range(layers)]
@@ -689,14 +707,18 @@ def ours_decode(args, w: W.Workload, world: int, rank: int, dev):
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
     if one_launch:
-        # the refresh is one kernel: mask and attention bytes over its time
+        # the refresh is one kernel (after the stages' launches, if any):
+        # mask and attention bytes over its time
         dom_bytes, dom_us = mask_bytes + attn_bytes[0], refresh_us
         dom_kernel = "mask_mma_kernel (mask + attention)"
         traffic = traffic_from_profile("mask_mma_kernel+attn", w.name)
+        if STAGES:
+            dom_kernel = "stage_score/stage_select + " + dom_kernel
+            traffic = None
     else:
         dom_bytes, dom_us = mask_bytes, mask_us
         dom_kernel = "mask_mma_kernel" if w.dtype != "f32" else "mask_fma_kernel"
-        traffic = traffic_from_profile(dom_kernel, w.name)
+        traffic = traffic_from_profile(dom_kernel, w.name) if not STAGES else None
     dom_gbs = dom_bytes / (dom_us * 1e-6) / 1e9
     roofline = {"bound": "hbm", "kernel": dom_kernel, "achieved": dom_gbs, "peak": hbm,
                 "peak_kind": f"{pk_kind} HBM copy", "unit": "GB/s", "frac": dom_gbs / hbm,
@@ -706,7 +728,7 @@ def ours_decode(args, w: W.Workload, world: int, rank: int, dev):
                         "split), algorithmic bytes over it" if rm > 1 or not one_launch else
                         "the step is this one launch: algorithmic bytes over the median step time")}
     step_gbs = step_bytes / (step_us * 1e-6) / 1e9
-    launches_refresh = 1 if one_launch else 2
+    launches_refresh = (1 if one_launch else 2) + stage_launches()
     launches_per_step = launches_refresh + (rm - 1)
 
     kern = {"how": "median timed step split by CUDA event-node intervals of one layer "
@@ -865,6 +887,7 @@ def ours_prefill(args, w: W.Workload, world: int, rank: int, dev, nested: bool):
     stream = torch.cuda.Stream(device=dev)
     code = {"bf16": hb.HIPS_BF16, "f32": hb.HIPS_F32, "e5m2": hb.HIPS_BF16_E5M2}[w.dtype]
     sess = hb.Session(dtype=code, flags=hb.FLAG_HEAD_MASKS if HEAD_MASKS else 0, stream=stream,
+                      stages=STAGES,
                       **layer_shape(w))
     lay.idxs = [sess.new_idx() for _ in range(layers)]
 
@@ -983,7 +1006,7 @@ def ours_prefill(args, w: W.Workload, world: int, rank: int, dev, nested: bool):
                     "us_per_layer": step_ms * 1e3},
         "timing": {"regions": len(regions), "region_ms_median": region_ms,
                    "region_ms_min": float(np.min(regions)), "region_ms_max": float(np.max(regions))},
-        "gpu_launches": 3 * steps,  # key-norm pre-pass, mask, attention
+        "gpu_launches": (3 + stage_launches()) * steps,  # key-norm pre-pass, mask, attention
         "clocks": clk.summary(),
     }
     if e2e:
@@ -994,9 +1017,11 @@ def ours_prefill(args, w: W.Workload, world: int, rank: int, dev, nested: bool):
 
 
 def main():
-    global HEAD_MASKS
+    global HEAD_MASKS, STAGES
     args = parse()
     HEAD_MASKS = args.head_masks
+    if args.stages:
+        STAGES = tuple(tuple(int(v) for v in st.split(":")) for st in args.stages.split(","))
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         # the oracle runs on rank 0's host cores alone; no process group
@@ -1007,7 +1032,7 @@ def main():
     try:
         line = ours(args, w, world, rank, local)
         if (args.workload == DEFAULT_WORKLOAD and not args.no_prefill and not HEAD_MASKS
-                and not args.two_calls):
+                and not args.two_calls and not STAGES):
             # the other half of the metric: prefill TFLOP/s, in the same line
             pw = W.PREFILL_32K
             pre = ours(args, pw, world, rank, local, nested=True)

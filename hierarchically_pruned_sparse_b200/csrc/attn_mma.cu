@@ -38,6 +38,16 @@ namespace hips {
 
 namespace {
 
+// 2^x by the SFU's ex2.approx.ftz instruction (relative error about 2^-22;
+// results below the normal range flush to 0, and 2^-inf = 0): one
+// instruction, where exp2f adds the handling of subnormal results that
+// softmax weights (at most 2^8, summed in fp32 and stored as bf16) never need.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 constexpr int kRows = 128;                 // query rows per MMA (M)
 constexpr int kHalves = 2;                 // MMA row halves per CTA
 constexpr int kCtaRows = kRows * kHalves;  // query rows per CTA
@@ -350,13 +360,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_mma_kernel(AttnArgs a) {
         const float nm = -m_ref;
 #pragma unroll
         for (int i = 0; i < kKeys; ++i) {
-          s[i] = exp2f(fmaf(s[i], a.scale_log2, nm));
+          s[i] = fast_exp2(fmaf(s[i], a.scale_log2, nm));
           ps4[i & 3] += s[i];
         }
       } else {
 #pragma unroll
         for (int i = 0; i < kKeys; ++i) {
-          s[i] = s[i] == -INFINITY ? 0.0f : exp2f(s[i] - m_ref);
+          s[i] = fast_exp2(s[i] - m_ref);  // 2^-inf = 0
           ps4[i & 3] += s[i];
         }
       }
