@@ -435,14 +435,95 @@ int cuda_status(cudaError_t e) {
   return HIPS_ERR_CUDA;
 }
 
+// Workspace bytes of one call with the kernels' own element types (0: no plan).
+size_t native_ws(const hips_params* params, int op) {
+  if (op == HIPS_OP_MASK) {
+    MaskPlan plan;
+    return plan_mask(params, 16, &plan) == HIPS_OK ? plan.ws : 0;
+  }
+  if (op == HIPS_OP_MASK_SPARSE) {  // either the fused launch or the two calls
+    const size_t m = native_ws(params, HIPS_OP_MASK);
+    const size_t s = native_ws(params, HIPS_OP_SPARSE);
+    return m && s ? std::max(m, s) : 0;
+  }
+  if (op == HIPS_OP_SPARSE || op == HIPS_OP_DENSE) {
+    AttnPlan plan;
+    return plan_attn(params, op == HIPS_OP_DENSE, &plan) == HIPS_OK ? plan.ws : 0;
+  }
+  return 0;
+}
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// ---------------------------------------------------------------- e5m2 by widening
+// e5m2 shapes that no e5m2 kernel plans (prefill query blocks, masks of more
+// than 16 query rows, attention of more than 8 rows per query block): the
+// keys (and values) a call reads, rows [0, seq_len) of every head, are
+// widened exactly to bf16 in the workspace, after the bf16 plan's own area,
+// and the bf16 kernels run on them. The e5m2 path is defined as the bf16 one
+// on the widened values, so the results are the same; the cost is one pass
+// over the cache and 2 bytes per element of workspace.
+hips_params bf16_view(const hips_params* p) {
+  hips_params b = *p;
+  b.dtype = HIPS_BF16;
+  b.kv_capacity = p->seq_len;  // the widened rows are compact
+  return b;
+}
+
+size_t widened_bytes(const hips_params* p, bool with_v) {
+  const size_t one = round256(static_cast<size_t>(p->batch) * p->n_kvheads * p->seq_len * hips::kD *
+                              sizeof(uint16_t));
+  return with_v ? 2 * one : one;
+}
+
+bool needs_widening(const hips_params* p, int op) {
+  return p->dtype == HIPS_BF16_E5M2 && native_ws(p, op) == 0;
+}
+
+// Widen k (and v) into the workspace; *b gets the bf16 view whose workspace
+// is the area before the widened rows, *kw and *vw the widened tensors.
+int widen_inputs(const void* k, const void* v, const hips_params* p, int op, hips_params* b,
+                 const void** kw, const void** vw) {
+  *b = bf16_view(p);
+  const size_t w = native_ws(b, op);
+  if (!w) return HIPS_ERR_UNSUPPORTED;
+  const bool with_v = v != nullptr;
+  const size_t off = round256(w);
+  if (!p->workspace || !aligned(p->workspace, 256) || p->workspace_bytes < off + widened_bytes(p, with_v))
+    return HIPS_ERR_WORKSPACE;
+  unsigned char* base = static_cast<unsigned char*>(p->workspace) + off;
+  const size_t one = widened_bytes(p, false);
+  cudaStream_t stream = static_cast<cudaStream_t>(p->stream);
+  const int64_t heads = static_cast<int64_t>(p->batch) * p->n_kvheads;
+  cudaError_t e = hips::launch_widen_e5m2(k, base, heads, p->seq_len, p->kv_capacity, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  *kw = base;
+  *vw = nullptr;
+  if (with_v) {
+    e = hips::launch_widen_e5m2(v, base + one, heads, p->seq_len, p->kv_capacity, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    *vw = base + one;
+  }
+  b->workspace_bytes = off;
+  return HIPS_OK;
+}
+
 int run_attention(const void* q, const void* k, const void* v, const int32_t* idx,
                   const hips_params* p, void* out, bool dense) {
-  int st = validate(p, dense ? HIPS_OP_DENSE : HIPS_OP_SPARSE);
+  const int op = dense ? HIPS_OP_DENSE : HIPS_OP_SPARSE;
+  int st = validate(p, op);
   if (st) return st;
   if (!q || !k || !v || !out || (!dense && !idx)) return HIPS_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       (idx && !aligned(idx, 4)))
     return HIPS_ERR_INVALID_ARG;
+  if (needs_widening(p, op)) {
+    hips_params b;
+    const void *kw, *vw;
+    st = widen_inputs(k, v, p, op, &b, &kw, &vw);
+    if (st) return st;
+    return run_attention(q, kw, vw, idx, &b, out, dense);
+  }
   AttnPlan plan;
   st = plan_attn(p, dense, &plan);
   if (st) return st;
@@ -621,20 +702,13 @@ int64_t hip_idx_row_stride(const hips_params* params) {
 
 size_t hip_workspace_size(const hips_params* params, int op) {
   if (validate(params, op) != HIPS_OK) return 0;
-  if (op == HIPS_OP_MASK) {
-    MaskPlan plan;
-    return plan_mask(params, 16, &plan) == HIPS_OK ? plan.ws : 0;
-  }
-  if (op == HIPS_OP_MASK_SPARSE) {  // either the fused launch or the two calls
-    const size_t m = hip_workspace_size(params, HIPS_OP_MASK);
-    const size_t s = hip_workspace_size(params, HIPS_OP_SPARSE);
-    return m && s ? std::max(m, s) : 0;
-  }
-  if (op == HIPS_OP_SPARSE || op == HIPS_OP_DENSE) {
-    AttnPlan plan;
-    return plan_attn(params, op == HIPS_OP_DENSE, &plan) == HIPS_OK ? plan.ws : 0;
-  }
-  return 0;
+  const size_t n = native_ws(params, op);
+  if (n || params->dtype != HIPS_BF16_E5M2) return n;
+  // e5m2 shapes no e5m2 kernel plans: the bf16 plan on widened rows
+  const hips_params b = bf16_view(params);
+  const size_t w = native_ws(&b, op);
+  if (!w) return 0;
+  return round256(w) + widened_bytes(params, op != HIPS_OP_MASK);
 }
 
 int hip_workspace_init(const hips_params* params) {
@@ -662,6 +736,13 @@ int hip_mask(const void* q, const void* k, const hips_params* params, int32_t* i
   if (st) return st;
   if (!q || !k || !idx_out) return HIPS_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx_out, 4)) return HIPS_ERR_INVALID_ARG;
+  if (needs_widening(params, HIPS_OP_MASK)) {
+    hips_params b;
+    const void *kw, *vw;
+    st = widen_inputs(k, nullptr, params, HIPS_OP_MASK, &b, &kw, &vw);
+    if (st) return st;
+    return hip_mask(q, kw, &b, idx_out);
+  }
   return launch_mask(q, k, params, idx_out, nullptr, nullptr);
 }
 
@@ -674,6 +755,13 @@ int hip_mask_sparse_attn(const void* q, const void* k, const void* v, const hips
       !aligned(idx_out, 4))
     return HIPS_ERR_INVALID_ARG;
   if (params->mask_len != params->seq_len) return HIPS_ERR_INVALID_ARG;  // a fresh mask
+  if (needs_widening(params, HIPS_OP_MASK_SPARSE)) {
+    hips_params b;
+    const void *kw, *vw;
+    st = widen_inputs(k, v, params, HIPS_OP_MASK_SPARSE, &b, &kw, &vw);
+    if (st) return st;
+    return hip_mask_sparse_attn(q, kw, vw, &b, idx_out, out);
+  }
   MaskPlan plan;
   st = plan_mask(params, 16, &plan, true);
   if (st) return st;

@@ -87,11 +87,16 @@ enum hips_status {
  * command of the SGLang pull request "[Feature] Support Efficient Sparse HiP
  * Attention (InfiniteHiP)"), while q and out are bf16. Every code widens
  * exactly to bf16, and the mask and attention are those of bf16 keys and
- * values with the widened values. Supported for masks of one query position
- * per mask row (decode, or b_q = 1) with at most 8 query rows, for masks of
- * 9 to 16 query rows with block_k <= 32 and topk / block_k <= 1024, and for
- * attention of at most 8 rows per query block; other shapes return
- * HIPS_ERR_UNSUPPORTED (from the call and as a zero hip_workspace_size). */
+ * values with the widened values. e5m2 kernels read the codes directly for
+ * masks of one query position per mask row (decode, or b_q = 1) with at most
+ * 8 query rows, for masks of 9 to 16 query rows with block_k <= 32 and
+ * topk / block_k <= 1024, and for attention of at most 8 rows per query
+ * block. Every other shape that bf16 supports (prefill query blocks, wider
+ * masks and attention) widens the keys (and values) it reads, rows [0,
+ * seq_len) of every head, into the workspace first and runs the bf16
+ * kernels on them: hip_workspace_size then includes 2 bytes per widened
+ * element (B x n_kvheads x seq_len x head_dim, once for a mask, twice when
+ * values are read), and the call makes one extra pass over the cache. */
 enum hips_dtype { HIPS_F32 = 0, HIPS_BF16 = 1, HIPS_BF16_E5M2 = 2 };
 
 enum hips_op { HIPS_OP_MASK = 0, HIPS_OP_SPARSE = 1, HIPS_OP_DENSE = 2, HIPS_OP_MASK_SPARSE = 3 };

@@ -137,27 +137,41 @@ def test_prefill_shapes_plan():
     assert hb.idx_row_stride(p) == 1 + 1024 + 64 + 544 + 1
 
 
-def test_e5m2_kv_plans_decode_and_rejects_other_shapes():
+def _up(n):
+    return (n + 255) // 256 * 256
+
+
+def test_e5m2_kv_plans_decode_natively_and_other_shapes_by_widening():
     f = 1 << 20
     p = _decode_params(dtype=hb.HIPS_BF16_E5M2)
     for op in (hb.OP_MASK, hb.OP_SPARSE, hb.OP_DENSE, hb.OP_MASK_SPARSE):
         assert hb.workspace_size(p, op) >= 256, op
     assert hb.mask_ptr(f, f, p, f) == hb.HIPS_ERR_WORKSPACE  # valid up to the missing workspace
+    # the decode shapes have e5m2 kernels: no room for widened rows
+    assert hb.workspace_size(p, hb.OP_MASK) < 8 * 131072 * 128 * 2
+
+    def widened(**kw):
+        # shapes without an e5m2 kernel: the bf16 plan (compact rows), then
+        # K (mask) or K and V (attention) widened to bf16 in the workspace
+        e = hb.params(**kw, dtype=hb.HIPS_BF16_E5M2)
+        b = hb.params(**kw, dtype=hb.HIPS_BF16)
+        rows = _up(kw["batch"] * kw["n_kvheads"] * kw["seq_len"] * 128 * 2)
+        for op, n in ((hb.OP_MASK, 1), (hb.OP_SPARSE, 2), (hb.OP_DENSE, 2), (hb.OP_MASK_SPARSE, 2)):
+            w = hb.workspace_size(b, op)
+            want = _up(w) + n * rows if w else 0  # no bf16 plan: none either
+            assert hb.workspace_size(e, op) == want, (op, hb.workspace_size(e, op), want)
+
     # more than 16 rows per mask (one MMA column block) has no e5m2 mask kernel
-    wide = _decode_params(dtype=hb.HIPS_BF16_E5M2, n_qheads=64, n_kvheads=2)
-    assert hb.workspace_size(wide, hb.OP_MASK) == 0
-    assert hb.mask_ptr(f, f, wide, f) == hb.HIPS_ERR_UNSUPPORTED
+    widened(batch=1, n_qheads=64, n_kvheads=2, seq_len=131072, q_len=1, q_pos0=131071,
+            block_q=1, block_k=2, topk=2048, sink=128, window=1024)
     # prefill query blocks: neither the mask nor the attention has an e5m2 kernel
-    pre = hb.params(batch=1, n_qheads=32, n_kvheads=8, seq_len=32768, q_len=32768, q_pos0=0,
-                    dtype=hb.HIPS_BF16_E5M2, block_q=64, block_k=2, topk=2048, sink=128,
-                    window=1024)
-    assert hb.workspace_size(pre, hb.OP_MASK) == 0
-    assert hb.workspace_size(pre, hb.OP_SPARSE) == 0
+    widened(batch=1, n_qheads=32, n_kvheads=8, seq_len=32768, q_len=32768, q_pos0=0,
+            block_q=64, block_k=2, topk=2048, sink=128, window=1024)
     # 2048 chunks per mask do not fit beside the tensor-core kernel's tiles:
     # e5m2 decode masks (one query position, at most 8 rows) then run on the
     # CUDA-core decode kernel, bf16 ones on the CUDA-core mask kernel
     big = _decode_params(dtype=hb.HIPS_BF16_E5M2, topk=4096)
-    assert hb.workspace_size(big, hb.OP_MASK) >= 256
+    assert 256 <= hb.workspace_size(big, hb.OP_MASK) < 8 * 131072 * 128 * 2
     assert hb.workspace_size(_decode_params(topk=4096), hb.OP_MASK) >= 256
 
 

@@ -8,10 +8,12 @@ must match the oracle's bit-exactly (the kernels select by canonical scores) and
 outputs stay within the bf16 tolerance. The e5m2 path must also give the
 same masks as the bf16 path run on the widened keys, and the one-launch
 decode the same outputs bit for bit (both attend in 64-key tiles in the same
-order).
+order). Shapes with no e5m2 kernel (prefill query blocks, attention of more
+than 8 rows per block) run on widened rows and are checked the same way.
 """
 import functools
 
+import numpy as np
 import pytest
 
 import oracle
@@ -95,25 +97,27 @@ def test_small_decode_shapes(w, fused):
     _check(w, fused)
 
 
-def test_sixteen_row_mask_and_no_sixteen_row_attention():
+def test_sixteen_row_mask_and_its_attention():
     # 16 rows per mask is the largest e5m2 mask (one MMA column block); the
-    # attention of more than 8 rows per query block has no e5m2 kernel
+    # attention of more than 8 rows per query block has no e5m2 kernel and
+    # runs on widened rows
     import torch
     from hierarchically_pruned_sparse_b200 import binding as hb
     w = W.Workload("e16", "decode", 1, 16, 1, 128, 2500, 1, 2, 64, 2, 8, "e5m2")
     x = _inputs(w)
-    kf, _ = pu.oracle_kv(x, w)
+    kf, vf = pu.oracle_kv(x, w)
     osh, bkw = pu.shapes(w)
     q, k, v = pu.torch_inputs(x, w)
     s = hb.Session(**bkw)
     idx = s.mask(q, k)
+    out = s.sparse_attn(q, k, v, idx)
     torch.cuda.synchronize()
     s.check()
     idx_ref, gap, _ = oracle.mask(x["q"][0], kf, osh)
-    pu.compare_masks(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref, gap,
-                     validate=pu.gpu_validator(x["q"][0], kf, osh, s, q, k))
-    with pytest.raises(hb.HipsError):
-        s.sparse_attn(q, k, v, idx)
+    ig = idx.cpu().numpy().reshape(idx_ref.shape)
+    pu.compare_masks(ig, idx_ref, gap, validate=pu.gpu_validator(x["q"][0], kf, osh, s, q, k))
+    ref = oracle.attention(x["q"][0], kf, vf, ig, osh)
+    pu.compare_outputs(out.float().cpu().numpy().reshape(ref.shape), ref, "e5m2")
 
 
 def test_reused_mask_with_appended_keys():
@@ -172,9 +176,32 @@ def test_dense_attention_over_e5m2():
     pu.compare_outputs(out.float().cpu().numpy().reshape(ref.shape), ref, "e5m2")
 
 
-def test_prefill_blocks_are_unsupported():
+# Shapes with no e5m2 kernel run on the bf16 kernels after the library widens
+# K and V exactly into the workspace (the e5m2 path is defined as the bf16 one
+# on the widened values): prefill query blocks, and attention of more than 8
+# rows per query block.
+PREFILL = W.Workload("e_pre", "prefill", 1, 8, 2, 128, 1000, 64, 2, 128, 16, 32, "e5m2")
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["one_call", "two_calls"])
+def test_prefill_blocks_by_widening(fused):
+    st = _check(PREFILL, fused)
+    assert st["rows"] == 2 * 16
+
+
+def test_dense_prefill_over_e5m2_by_widening():
+    import torch
     from hierarchically_pruned_sparse_b200 import binding as hb
-    p = hb.params(batch=1, n_qheads=4, n_kvheads=1, seq_len=512, q_len=512, q_pos0=0,
-                  dtype=hb.HIPS_BF16_E5M2, block_q=64, block_k=2, topk=64)
-    assert hb.workspace_size(p, hb.OP_MASK) == 0
-    assert hb.mask_ptr(1 << 20, 1 << 20, p, 1 << 20) == hb.HIPS_ERR_UNSUPPORTED
+    x = _inputs(PREFILL)
+    kf, vf = pu.oracle_kv(x, PREFILL)
+    osh, bkw = pu.shapes(PREFILL)
+    q, k, v = pu.torch_inputs(x, PREFILL)
+    s = hb.Session(**bkw)
+    out = torch.empty_like(q)
+    hb.hip_dense_attn(q, k, v, s.p, out)
+    torch.cuda.synchronize()
+    s.check()
+    rows = np.arange(0, q.numel() // 128, 7)  # every 7th (head, position) row
+    ref = oracle.attention(x["q"][0], kf, vf, None, osh, rows=rows)
+    got = out.float().cpu().numpy().reshape(-1, 128)[rows]
+    pu.compare_outputs(got, ref, "e5m2")
