@@ -10,6 +10,7 @@
 #include "hip_sparse.h"
 #include "hips_common.cuh"
 #include "hips_kernels.h"
+#include "widen.h"
 
 static_assert(HIPS_F32 == hips::kDtypeF32 && HIPS_BF16 == hips::kDtypeBf16 &&
                   HIPS_BF16_E5M2 == hips::kDtypeBf16E5m2,

@@ -127,11 +127,6 @@ int decode_smem_bytes(MaskArgs& a, bool attend, int smem_cap);
 int decode_max_active_clusters(const MaskArgs& a, int smem);
 cudaError_t launch_decode(const MaskArgs& a, int smem, cudaStream_t stream);
 
-// Exact widening of e5m2 K or V rows [0, rows) of `heads` heads (head stride
-// src_cap rows) into compact bf16 rows (head stride `rows`) (widen.cu).
-cudaError_t launch_widen_e5m2(const void* src, void* dst, int64_t heads, int64_t rows, int64_t src_cap,
-                              cudaStream_t stream);
-
 // Pruning stages (stages.cu). A stage of a mask row ranks at most
 // kStageMaxChunks chunks (the selection keeps their score keys in shared
 // memory).

@@ -8,6 +8,7 @@
 
 #include "hips_common.cuh"
 #include "hips_kernels.h"
+#include "widen.h"
 
 namespace hips {
 namespace {
