@@ -244,6 +244,13 @@ def test_bad_stage_schedules_are_rejected(stages):
     assert hb.workspace_size(p, hb.OP_SPARSE) > 0  # the attention does not read them
 
 
+def test_a_stage_count_without_a_stage_array_is_rejected():
+    p = _decode_params()
+    p.n_stages = 2  # and no array
+    assert hb.workspace_size(p, hb.OP_MASK) == 0
+    assert hb.mask_ptr(1 << 20, 1 << 20, p, 1 << 20) == hb.HIPS_ERR_INVALID_ARG
+
+
 def test_stage_schedules_that_leave_more_than_n0_chunks_are_unsupported():
     # the iteration starts from at most topk / block_k = 1024 chunks: 8-key
     # chunks that all survive (16384 of them at 128k keys) are too many, so

@@ -89,3 +89,20 @@ def test_layer_buffers_outgrow_the_l2_by_the_bytes_a_step_touches():
     # prefill reads all of q, k and v; a requested count is kept
     assert bench.touched_bytes(W.PREFILL_32K) == (2 * 8 + 32) * 32768 * 128 * 2
     assert bench.layer_count(W.PREFILL_32K, 400 << 20, 5) == 5
+
+
+def test_stage_launch_counts():
+    # a scoring and a selection launch per stage that ranks; one selection
+    # launch (cut and halve only) when none ranks; nothing without stages
+    saved = bench.STAGES
+    try:
+        bench.STAGES = ()
+        assert bench.stage_launches() == 0
+        bench.STAGES = ((128, 0, 4), (32, 32768, 4), (8, 8192, 1))
+        assert bench.stage_launches() == 4
+        bench.STAGES = ((64, 0, 1),)
+        assert bench.stage_launches() == 1
+        cfg = bench.config_of(W.DECODE_128K, 0)
+        assert cfg["stages"] == [{"chunk_size": 64, "stage_k": None, "stride_q": 1}]
+    finally:
+        bench.STAGES = saved
