@@ -28,18 +28,20 @@
 //    ranks. Per chunk it reads b_k d-element rows: a gather bound by HBM,
 //    spread over every SM.
 //  * stage_select: one CTA per mask row, with the row's score keys staged in
-//    shared memory (all loads in flight at once). An exact radix select
-//    (four 8-bit
-//    digits of the order-preserving key of the score, most significant
-//    first) finds the keep-th largest score; chunks above it are kept, and
-//    of those equal to it the lowest-indexed (lists are in start order, so
-//    the lowest start) fill the rest. An order-preserving scan (each warp a
-//    contiguous run, 32 consecutive chunks at a time) places the ties' ranks
-//    and then the kept chunks' pieces (the next stage's chunks) in start
-//    order. A final list
-//    is then halved in shared memory for as long as the halves number at
-//    most n0 (the iteration's rounds that keep every candidate and so need
-//    no scores).
+//    shared memory (all loads in flight at once). A histogram of 2048
+//    buckets linear in the score over [min, max] finds the bucket of the
+//    keep-th largest score (a bucket above another holds only larger
+//    scores); chunks above it are kept, and its members (a handful) are
+//    ranked exactly by (score desc, index asc) -- lists are in start order,
+//    so the lowest start wins a tie. A cut bucket of more than 2048 members
+//    (heavy ties) falls back to an exact radix select over four 8-bit digits
+//    of the order-preserving key. An order-preserving scan (each warp a
+//    contiguous run, 32 consecutive chunks at a time) lists the kept chunks
+//    in start order; every input chunk but the last has the input
+//    granularity, so their pieces (the next stage's chunks) are placed
+//    without a scan. A final list is then halved in shared memory for as
+//    long as the halves number at most n0 (the iteration's rounds that keep
+//    every candidate and so need no scores).
 #include <cuda_runtime.h>
 
 #include <algorithm>
