@@ -129,3 +129,36 @@ def test_decode_128k_pr_schedule_one_launch():
 
 def test_decode_128k_pr_schedule_two_calls():
     _check(W.DECODE_128K, PR_LIKE_128K, False)
+
+
+@pytest.mark.parametrize("stages", [((4, 1024, 1),), ((2, 2048, 1),)],
+                         ids=["ties_in_one_bucket", "ties_past_the_bucket_band"])
+def test_equal_keys_keep_the_lowest_starts(stages):
+    # every key row is the same, so every score ties: each stage and round
+    # keeps the chunks with the lowest starts. 2048 tied chunks are ranked
+    # in the selection's cut bucket; 4096 exceed its band and take the
+    # digit-by-digit selection instead.
+    import torch
+    from hierarchically_pruned_sparse_b200 import binding as hb
+    T, d = 8192, 128
+    rng = np.random.default_rng(9)
+    qf = rng.standard_normal((1, 1, 1, d)).astype(np.float32)
+    row = rng.standard_normal(d).astype(np.float32)
+    kf = np.ascontiguousarray(np.broadcast_to(row, (1, 1, T, d)))
+    vf = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(torch.bfloat16)  # noqa: E731
+    q, k, v = to(qf), to(kf), to(vf)
+    qb, kb, vb = (x.float().cpu().numpy() for x in (q, k, v))
+    common = dict(batch=1, n_qheads=1, n_kvheads=1, seq_len=T, q_len=1, q_pos0=T - 1,
+                  block_q=1, block_k=1, topk=1024)
+    s = hb.Session(dtype=hb.HIPS_BF16, stages=stages, **common)
+    idx, out = s.mask_sparse_attn(q, k, v)
+    torch.cuda.synchronize()
+    s.check()
+    osh = oracle.shape(head_dim=d, stages=stages, **common)
+    idx_ref, gap, _ = oracle.mask(qb, kb, osh)
+    got = idx.cpu().numpy().reshape(idx_ref.shape)
+    assert list(idx_ref[0, 1:1 + idx_ref[0, 0]]) == list(range(1024))
+    np.testing.assert_array_equal(got, idx_ref)
+    ref = oracle.attention(qb, kb, vb, got, osh)
+    pu.compare_outputs(out.float().cpu().numpy().reshape(ref.shape), ref, "bf16")
