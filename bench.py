@@ -726,6 +726,8 @@ def ours_decode(args, w: W.Workload, world: int, rank: int, dev):
                 "time_us": dom_us,
                 "how": ("the refresh step's share of the median timed step (event-node "
                         "split), algorithmic bytes over it" if rm > 1 or not one_launch else
+                        "the step is the stage launches and this one launch: algorithmic bytes "
+                        "over the median step time" if STAGES else
                         "the step is this one launch: algorithmic bytes over the median step time")}
     step_gbs = step_bytes / (step_us * 1e-6) / 1e9
     launches_refresh = (1 if one_launch else 2) + stage_launches()
@@ -734,7 +736,7 @@ def ours_decode(args, w: W.Workload, world: int, rank: int, dev):
     kern = {"how": "median timed step split by CUDA event-node intervals of one layer "
                    "(replays outside the timed region), scaled to the step",
             "step_call": "hip_mask + hip_sparse_attn" if two else "hip_mask_sparse_attn",
-            "one_launch": one_launch, "scored_candidates": scored,
+            "one_launch": one_launch and not STAGES, "scored_candidates": scored,
             "mask_bytes": mask_bytes, "attn_bytes": attn_bytes[0]}
     if one_launch:
         kern["refresh_us"] = refresh_us
