@@ -258,3 +258,28 @@ def test_stage_schedules_that_leave_more_than_n0_chunks_are_unsupported():
     assert hb.workspace_size(_decode_params(stages=((8, 0, 1),)), hb.OP_MASK) == 0
     assert hb.workspace_size(_decode_params(stages=((8, 16384, 1),)), hb.OP_MASK) == 0
     assert hb.workspace_size(_decode_params(stages=((8, 8192, 1),)), hb.OP_MASK) > 0
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    # sizes and field offsets of hips_params and hips_stage as a C compiler
+    # lays them out from include/hip_sparse.h, against the ctypes mirrors
+    import ctypes
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    fields = [f for f, _ in hb.Params._fields_]
+    sfields = [f for f, _ in hb.Stage._fields_]
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "hip_sparse.h"', 'int main(void) {',
+             '  printf("%zu %zu\\n", sizeof(hips_params), sizeof(hips_stage));']
+    lines += [f'  printf("%zu\\n", offsetof(hips_params, {f}));' for f in fields]
+    lines += [f'  printf("%zu\\n", offsetof(hips_stage, {f}));' for f in sfields]
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", f"-I{os.path.join(root, 'include')}", str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    vals = [int(v) for v in out]
+    assert vals[0] == ctypes.sizeof(hb.Params) and vals[1] == ctypes.sizeof(hb.Stage)
+    assert vals[2:2 + len(fields)] == [getattr(hb.Params, f).offset for f in fields]
+    assert vals[2 + len(fields):] == [getattr(hb.Stage, f).offset for f in sfields]
